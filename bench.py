@@ -1,0 +1,391 @@
+"""Benchmark of the fused grouped W4A16 MoE layer on B200.
+
+Default workload (one "step"): one decode step of a 16-layer stack of
+OLMoE-shaped MoE layers (hidden 2048, expert intermediate 1024, 64 SwiGLU
+experts, top-8; int4 group-128 experts, all resident, 3.32 GB packed) at
+T=16 tokens, with the residual x + MoE(x) between layers. Every step runs
+route -> group -> grouped W4A16 FFN -> combine for each layer through the
+library's C ABI, replayed from one CUDA graph. The same step is also timed at
+T = 1, 4, 64 (the rest of the decode sweep) and reported under "sweep".
+
+metric: MoE-layer tokens/s = T * layers / step time (device time, CUDA events).
+e2e:    the same metric with the activations copied host->device from pinned
+        memory before and the output copied back after, inside the timed region.
+roofline: the grouped FFN (gate/up + down kernels) per layer call: algorithmic
+        bytes = active experts x 3,244,032 B of packed codes + scales, over the
+        call's CUDA-event duration, against the measured HBM copy bandwidth.
+cpu_baseline: the CPU oracle (numpy, fp64) on a bounded sample of the workload.
+
+--impl reference runs that oracle as the reference arm (rank 0 only).
+Multi-GPU: replicas only (each rank runs the whole workload on its own GPU;
+the layer has no exchange step), timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+H, I, E, K, LAYERS = 2048, 1024, 64, 8, 16
+SWEEP_T = (1, 4, 16, 64)
+METRIC = "MoE-layer tokens/s; HBM GB/s (decode) and TC TFLOP/s (prefill) vs B200 peak"
+REC_BYTES = 3 * I * H // 2 + 3 * (I * H // 128) * 2   # one packed expert record
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--T", type=int, default=16)
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc"])
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        import torch
+        self.idx = str(device_index)
+        try:  # the UUID names the same GPU whatever CUDA_VISIBLE_DEVICES says
+            u = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.idx = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            pass
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- the stack
+
+class Stack:
+    """16 OLMoE-shaped layers: per layer a packed expert bank and a router, plus
+    per-T buffers. Weights are drawn on the device with the seeded recipe."""
+
+    def __init__(self, layers, path):
+        import torch
+
+        import synth
+        import w4a16_mixture_experts_moe_b200 as M
+        from w4a16_mixture_experts_moe_b200.layer import ExpertBank
+        self.M, self.torch, self.layers = M, torch, layers
+        self.path = {"auto": M.MOE_PATH_AUTO, "gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC}[path]
+        self.banks, self.routers = [], []
+        for l in range(layers):
+            gate, up, down = synth.expert_bank(l, E, H, I, device="cuda")
+            bank = ExpertBank(E, H, I)
+            bank.pack(gate, up, down)
+            del gate, up, down
+            self.banks.append(bank)
+            self.routers.append(synth.router_weight(l, E, H, device="cuda"))
+        torch.cuda.synchronize()
+
+    def buffers(self, T):
+        from w4a16_mixture_experts_moe_b200.layer import LayerBuffers
+        torch = self.torch
+        bufs = [LayerBuffers(T, K, E, H, I, path=self.path) for _ in range(self.layers)]
+        xs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        return bufs, xs
+
+    def forward(self, bufs, xs, x_in, events=None):
+        """x_in -> layer 0 -> ... -> returns the output buffer. events: optional
+        list of (start, end) CUDA events recorded around each layer's FFN call."""
+        from w4a16_mixture_experts_moe_b200.layer import moe_layer_forward
+        M = self.M
+        cur = x_in
+        for l in range(self.layers):
+            out = xs[l % 2] if cur is not xs[l % 2] else xs[(l + 1) % 2]
+            b = bufs[l]
+            T = b.T
+            if events is None:
+                moe_layer_forward(cur, self.routers[l], self.banks[l], b, residual=cur, out=out)
+            else:
+                M.moe_route_topk(cur, self.routers[l], T, H, E, K, None, 0, b.logits, b.topk_ids, b.topk_w)
+                M.moe_group_tokens(b.topk_ids, T, K, E, b.counts, b.offsets, b.sorted_pair, b.pair_pos,
+                                   b.group_ws, b.group_ws_bytes)
+                events[l][0].record()
+                M.moe_grouped_w4a16_ffn(cur, b.sorted_pair, b.offsets, self.banks[l].ptr, self.banks[l].rec, None,
+                                        E, T, K, E, H, I, b.path, b.y, b.ffn_ws, b.ffn_ws_bytes)
+                events[l][1].record()
+                M.moe_combine(b.y, b.topk_w, b.pair_pos, cur, T, K, H, out)
+            cur = out
+        return cur
+
+
+def time_graph(torch, graph, steps, warmup):
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        graph.replay()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def measure_T(stack, T, steps, warmup, world, want_e2e=True, want_roofline=True):
+    """Device-timed step, e2e step and per-call FFN timing at T tokens."""
+    import synth
+    torch, M = stack.torch, stack.M
+    bufs, xs = stack.buffers(T)
+    x_dev = synth.activations(T, H, device="cuda")
+    x_host = synth.activations(T, H).pin_memory()
+    out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    x_in = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    x_in.copy_(x_dev)
+
+    # eager warm-up (also loads kernels before capture)
+    stack.forward(bufs, xs, x_in)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    launches0 = M.moe_launch_counter()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        y = stack.forward(bufs, xs, x_in)
+    launches_per_step = M.moe_launch_counter() - launches0
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        x_in.copy_(x_host, non_blocking=True)
+        y2 = stack.forward(bufs, xs, x_in)
+        out_host.copy_(y2, non_blocking=True)
+    torch.cuda.synchronize()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms = time_graph(torch, g, steps, warmup)
+    barrier(world)
+    ms = max_over_ranks(ms, world)
+    res = {"T": T, "ms_per_step": ms, "launches_per_step": int(launches_per_step), "clocks": clk.summary()}
+    if want_e2e:
+        barrier(world)
+        ms_e2e = max_over_ranks(time_graph(torch, g2, steps, warmup), world)
+        res["ms_e2e"] = ms_e2e
+    if want_roofline:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(stack.layers)]
+        per_call = []
+        reps = max(3, min(steps, 10))
+        for r in range(reps + 2):
+            stack.forward(bufs, xs, x_in, events=ev)
+            torch.cuda.synchronize()
+            if r >= 2:
+                per_call += [a.elapsed_time(b) for a, b in ev]
+        n_act = [int((b.counts > 0).sum().item()) for b in bufs]
+        res["ffn_ms_per_call"] = statistics.mean(per_call)
+        res["n_active_mean"] = statistics.mean(n_act)
+        res["ffn_bytes_per_call"] = statistics.mean(n_act) * REC_BYTES
+    del g, g2
+    return res
+
+
+# ----------------------------------------------------------------------------- CPU oracle (baseline / reference)
+
+def oracle_sample(T, reps):
+    """Time the oracle on `reps` passes of one OLMoE layer at T tokens.
+    Returns (layer-tokens per second, cores, description). Quantisation (an
+    offline step on both sides) is done before the clock starts."""
+    import numpy as np
+    import torch
+
+    import synth
+    from oracle import exactmoe_oracle as o
+    from threadpoolctl import threadpool_info
+    gate, up, down = synth.expert_bank(0, E, H, I, device="cuda" if torch.cuda.is_available() else "cpu")
+    g, u, d = gate.cpu(), up.cpu(), down.cpu()
+    del gate, up, down
+    packs = [[o.quantize_pack(m[e].double().numpy()) for e in range(E)] for m in (g, u, d)]
+    arrays = []
+    for m in packs:
+        arrays.append(np.stack([p for p, _ in m]))
+        arrays.append(np.stack([s for _, s in m]))
+    wr = synth.router_weight(0, E, H).double().numpy()
+    x = synth.activations(T, H).double().numpy()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        experts = o.PackedExperts(*arrays)       # fresh: dequantisation is part of the timed work
+        o.moe_layer(x, wr, experts, K, residual=x)
+    dt = time.perf_counter() - t0
+    cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return T * reps / dt, cores, f"{reps} pass(es) of layer 0 of the stack at T={T} (dequant + router + top-k + " \
+                                 f"grouping + FFN + combine; quantisation not timed), {dt:.1f} s"
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    reps = max(1, a.steps // 10)
+    v, cores, desc = oracle_sample(a.T, reps)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "layer-tokens/s", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * a.T * a.layers / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"olmoe-{a.layers}L-decode", "T": a.T, "layers": a.layers, "H": H, "I": I,
+                       "E": E, "k": K},
+            "cpu_baseline": {"value": v, "unit": "layer-tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "layer-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+        return
+    import torch
+    rank, world, local = dist_setup(a.gpus)
+    P = peaks()
+    stack = Stack(a.layers, a.path)
+    head = measure_T(stack, a.T, a.steps, a.warmup, world)
+    sweep = {}
+    if not a.no_sweep:
+        for T in SWEEP_T:
+            if T == a.T:
+                r = head
+            else:
+                r = measure_T(stack, T, a.steps, a.warmup, world, want_e2e=False)
+            sweep[str(T)] = {"value": T * a.layers / (r["ms_per_step"] / 1e3) * world,
+                             "ms_per_step": r["ms_per_step"],
+                             "ffn_hbm_frac": (r["ffn_bytes_per_call"] / (r["ffn_ms_per_call"] / 1e3) / 1e9)
+                             / P["hbm_gbs"],
+                             "n_active_mean": r["n_active_mean"]}
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        v, cores, desc = oracle_sample(a.T, 2)
+        cpu = {"value": v, "unit": "layer-tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    if rank == 0:
+        T, L = a.T, a.layers
+        value = T * L * world / (head["ms_per_step"] / 1e3)
+        achieved = head["ffn_bytes_per_call"] / (head["ffn_ms_per_call"] / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "layer-tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"olmoe-{L}L-decode", "T": T, "layers": L, "H": H, "I": I, "E": E, "k": K,
+                       "weights": "int4 group-128 symmetric, all experts resident",
+                       "l2": "inputs larger than L2 (3.32 GB of packed experts read per step)",
+                       "parallelism": f"replicas{world}"},
+            "e2e": {"value": T * L * world / (head["ms_e2e"] / 1e3), "unit": "layer-tokens/s",
+                    "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
+            "roofline": {"bound": "hbm", "kernel": "moe_grouped_w4a16_ffn (gate/up + down kernels), per layer call",
+                         "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / P["hbm_gbs"], "traffic": None,
+                         "peak_source": P["source"], "bytes_per_call": head["ffn_bytes_per_call"],
+                         "ms_per_call": head["ffn_ms_per_call"]},
+            "cpu_baseline": cpu,
+            "gpu_launches": head["launches_per_step"] * a.steps,
+            "clocks": head["clocks"],
+            "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,270 @@
+/*
+ * exactmoe.h — C ABI of the fused grouped W4A16 routed-expert MoE layer.
+ *
+ * Method: "Every Expert Counts: ExactMoE for Memory-Efficient W4A16 Inference"
+ * (A. Saab, arXiv 2608.15383). The Abstract fixes symmetric group-128 four-bit
+ * quantisation of the routed experts only, a BF16 router with an unchanged
+ * top-k procedure, and fused grouped MoE kernels fed by a GPU-resident expert
+ * slot cache over pinned host memory. The Figure 1 caption fixes the order of
+ * the steps: pack once; the BF16 router selects experts; tokens are grouped by
+ * selected expert; the active experts run in fused grouped kernels; cache
+ * misses move packed weights and scales without materialising FP16 experts.
+ *
+ * Conventions for every entry point below:
+ *  - Pointers are DEVICE pointers unless a parameter says "host". The caller
+ *    owns every buffer; no hot-path call allocates device memory. Scratch
+ *    space is passed in as a workspace whose size the *_workspace_size
+ *    functions return.
+ *  - BF16 values travel as raw 16-bit patterns (moe_bf16).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream) and never synchronise, except moe_read_device_error.
+ *  - Every call returns MOE_OK or an error status; moe_last_error() gives a
+ *    message for the calling host thread. A failed argument check launches
+ *    nothing. Errors found on the device (an expert id out of range, an expert
+ *    that is not resident) are written to the first word of the workspace and
+ *    read back with moe_read_device_error.
+ *  - Shapes: hidden H and expert intermediate I are multiples of 128 (the
+ *    quantisation group); 1 <= E <= 256 experts; 1 <= k <= min(E, 32).
+ *
+ * Packed weight format (defined by this library; the pages' MARLIN format is
+ * prior art for a different GPU): for an nn.Linear weight W[N][K] (out x in),
+ *  - scale s[n][g] = bf16_rn(absmax(W[n][128g .. 128g+127]) / 7), fp32 divide;
+ *  - code q[n][k] = clamp(rint(W[n][k] / s[n][k/128]), -8, 7), fp32 divide,
+ *    ties to even, q = 0 where s = 0; stored offset-binary u = q + 8;
+ *  - row n of the packed matrix is K/2 bytes = K/8 little-endian 32-bit words;
+ *    word j holds k in [8j, 8j+8), with k = 8j + 2i + h (i = 0..3, h = 0..1)
+ *    at bits [4(i + 4h), 4(i + 4h) + 4). Shifting a word right by 4i and
+ *    masking 0x000F000F yields the codes of k = 8j+2i and 8j+2i+1 in the two
+ *    16-bit halves, which is what the kernels' in-register dequant consumes;
+ *  - scales are row-major [N][K/128] BF16.
+ * One expert is one record: gate [I][H/2], up [I][H/2], down [H][I/2] packed
+ * bytes, then the gate, up and down scales (moe_expert_record_layout gives
+ * the offsets). A bank is an array of records with a fixed stride; a slot is
+ * one record of a bank.
+ */
+#ifndef EXACTMOE_H
+#define EXACTMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;   /* raw BF16 bit pattern */
+typedef void *moe_stream_t;  /* a cudaStream_t */
+
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad flag, buffer too small */
+  MOE_ERR_SHAPE = 2,       /* shape outside the supported range */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+  MOE_ERR_CAPACITY = 4,    /* more distinct experts than cache slots */
+  MOE_ERR_DEVICE = 5,      /* a kernel flagged bad data (see device codes) */
+  MOE_ERR_UNSUPPORTED = 6  /* no path for this request on this device */
+};
+
+/* Device error codes written to workspace word 0 (first writer wins). */
+enum {
+  MOE_DEVERR_NONE = 0,
+  MOE_DEVERR_EXPERT_ID = 1,   /* a top-k id outside [0, E) */
+  MOE_DEVERR_NOT_RESIDENT = 2,/* an active expert has no valid slot */
+  MOE_DEVERR_TIMEOUT = 3      /* a bounded pipeline wait ran out */
+};
+
+/* Message for the last failed call on this host thread ("" if none). */
+const char *moe_last_error(void);
+
+/* ABI version, bumped on any incompatible change. */
+int moe_abi_version(void);
+
+/* Number of kernels this library has enqueued in this process (a host-side
+ * count taken at each launch site; a CUDA graph captured from these calls
+ * replays its kernels without counting again). */
+uint64_t moe_launch_counter(void);
+
+/* Byte offsets of the six parts of one expert record, and its size.
+ * All offsets are multiples of 256 bytes. */
+typedef struct {
+  int64_t gate_q, up_q, down_q; /* packed codes */
+  int64_t gate_s, up_s, down_s; /* BF16 scales */
+  int64_t bytes;                /* record size */
+} moe_record_layout;
+
+int moe_expert_record_layout(int H, int I, moe_record_layout *out);
+
+/*
+ * A1 — quantise and pack (Abstract: symmetric group-128 int4 weights for the
+ * routed experts; Figure 1 caption: packed once, offline).
+ *   w       [E][N][K] BF16, one nn.Linear weight per expert (K = in).
+ *   packed  expert e's codes at packed + e*packed_stride, [N][K/2] bytes.
+ *   scales  expert e's scales at (char*)scales + e*scales_stride, [N][K/128].
+ * Strides are in bytes (packed a multiple of 4, scales of 2; ignored when
+ * E == 1), so the output can land directly in the records of a bank.
+ * w must be 8-byte, packed 4-byte and scales 2-byte aligned. K % 128 == 0,
+ * N >= 1. Bit-exact with the format defined above.
+ */
+int moe_quantize_pack(const moe_bf16 *w, int E, int N, int K,
+                      uint8_t *packed, int64_t packed_stride,
+                      moe_bf16 *scales, int64_t scales_stride,
+                      moe_stream_t stream);
+
+/* Flags of moe_route_topk. */
+#define MOE_RENORM 1       /* divide the k weights by their sum */
+#define MOE_LOGITS_GIVEN 2 /* read `logits` instead of computing them */
+#define MOE_IDS_GIVEN 4    /* read `topk_ids`, only produce their weights */
+
+/*
+ * A2 + A3 — BF16 router logits, full softmax and unchanged top-k
+ * (Abstract: the router stays BF16 and the top-k routing procedure is
+ * unchanged; Figure 1 caption: the original BF16 router selects experts).
+ *   x         [T][H] BF16 activations.
+ *   w_router  [E][H] BF16 (nn.Linear convention).
+ *   bias      [E] fp32 added to the logits before softmax/top-k, or NULL.
+ *   logits    [T][E] BF16: written (fp32 sum rounded to BF16), or read when
+ *             MOE_LOGITS_GIVEN is set.
+ *   topk_ids  [T][k] int32: the k largest keys fp32(logit)+bias (NaN counts
+ *             as -inf), ties to the lower index, ordered by descending key
+ *             then ascending index. Read instead when MOE_IDS_GIVEN is set
+ *             (ids outside [0, E) get weight 0; moe_group_tokens flags them).
+ *   topk_w    [T][k] fp32: softmax probabilities (over all E) of the ids,
+ *             renormalised over the k when MOE_RENORM is set.
+ * T may be 0 (no launch).
+ */
+int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router,
+                   int T, int H, int E, int k,
+                   const float *bias, int flags,
+                   moe_bf16 *logits, int32_t *topk_ids, float *topk_w,
+                   moe_stream_t stream);
+
+/*
+ * A4 — group the T*k (token, slot) pairs by expert (Figure 1 caption: tokens
+ * are grouped by selected expert).
+ *   topk_ids    [T][k] int32.
+ *   counts      [E] int32 pairs per expert.
+ *   offsets     [E+1] int32 exclusive prefix sum of counts.
+ *   sorted_pair [T*k] int32 flat pair indices p = t*k + j, ordered by expert
+ *               and, within an expert, by p (a stable counting sort; the
+ *               result is unique and deterministic).
+ *   pair_pos    [T*k] int32 inverse: sorted_pair[pair_pos[p]] == p; -1 for a
+ *               pair whose id is out of range (also flagged on the device).
+ *   ws          workspace of at least moe_group_workspace_size(T, k, E) bytes,
+ *               256-byte aligned. Word 0 is the device error word; this call
+ *               clears it first.
+ */
+size_t moe_group_workspace_size(int T, int k, int E);
+int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E,
+                     int32_t *counts, int32_t *offsets,
+                     int32_t *sorted_pair, int32_t *pair_pos,
+                     void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* FFN execution paths. */
+#define MOE_PATH_AUTO 0 /* chosen from the average rows per expert, T*k/E */
+#define MOE_PATH_GEMV 1 /* decode-sized groups: weight-streaming, HBM-bound */
+#define MOE_PATH_TC 2   /* prefill-sized groups: tcgen05 tensor cores */
+
+/*
+ * A5 + A6 — the grouped SwiGLU expert FFN with in-kernel int4 dequantisation
+ * (Abstract: fused grouped MoE kernels over W4A16 experts; Figure 1 caption:
+ * packed weights and scales are consumed without materialising FP16 experts).
+ * For sorted row r of expert e (offsets[e] <= r < offsets[e+1]) and token
+ * t = sorted_pair[r] / k:
+ *   h[r] = bf16_rn(silu(x[t] Wg_e^T) * (x[t] Wu_e^T))      (fp32 sums)
+ *   y[r] = bf16_rn(h[r] Wd_e^T)                             (fp32 sums)
+ *   x            [T][H] BF16.
+ *   bank         device array of expert records with stride record_bytes
+ *                (moe_expert_record_layout(H, I).bytes or larger, multiple
+ *                of 256).
+ *   expert_slot  [E] int32 record index of each expert in the bank, or NULL
+ *                for the identity (record e holds expert e). An active
+ *                expert whose slot is outside [0, n_slots) is skipped and
+ *                flagged (MOE_DEVERR_NOT_RESIDENT).
+ *   y            [T*k][H] BF16, rows in sorted order.
+ *   ws           at least moe_ffn_workspace_size(T, k, E, H, I, path) bytes,
+ *                256-byte aligned; holds the error word and h.
+ * The GEMV path applies each group's scale to the fp32 partial sum of q*x
+ * over that group; the tensor-core path dequantises q*s to BF16 (one
+ * rounding) before the MMA.
+ */
+size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path);
+int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair,
+                          const int32_t *offsets, const void *bank,
+                          int64_t record_bytes, const int32_t *expert_slot,
+                          int n_slots, int T, int k, int E, int H, int I,
+                          int path, moe_bf16 *y, void *ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/*
+ * A7 — router-weighted combine (implied by the MoE layer; the pages do not
+ * spell it out):
+ *   out[t] = bf16_rn(residual[t] + sum_{j=0..k-1} topk_w[t][j] * y[pair_pos[t*k+j]])
+ * summed in fp32 in increasing j. residual may be NULL (zero); pairs with
+ * pair_pos < 0 contribute nothing. out may alias residual.
+ */
+int moe_combine(const moe_bf16 *y, const float *topk_w,
+                const int32_t *pair_pos, const moe_bf16 *residual,
+                int T, int k, int H, moe_bf16 *out, moe_stream_t stream);
+
+/*
+ * Synchronises `stream`, reads the device error word of a workspace written
+ * by moe_group_tokens or moe_grouped_w4a16_ffn, clears it, and returns
+ * MOE_OK or MOE_ERR_DEVICE (the code is stored in *code if code != NULL).
+ */
+int moe_read_device_error(void *ws, moe_stream_t stream, int32_t *code);
+
+/*
+ * A8 — GPU-resident expert slot cache over a pinned host pool (Abstract: a
+ * configurable GPU-resident slot cache over experts kept in pinned host
+ * memory; Figure 1 caption: the pinned pool keeps every packed expert and a
+ * miss moves packed weights and scales; Figure 2 caption: with capacity
+ * >= E every expert is resident and lookup accounting is bypassed).
+ *
+ * The cache owns only host bookkeeping (an LRU per layer) and two CUDA
+ * events per layer; all memory is the caller's:
+ *   pinned_pool   host, page-locked, [layers][E] records of record_bytes.
+ *   device_slots  device, [layers][slots] records of record_bytes.
+ *   expert_slot   device, [layers][E] int32, the table the FFN reads
+ *                 (-1 = not resident). slot_cache_fill keeps it current.
+ */
+typedef struct moe_slot_cache moe_slot_cache;
+
+int slot_cache_create(moe_slot_cache **out, int layers, int E, int slots,
+                      int64_t record_bytes, const void *pinned_pool,
+                      void *device_slots, int32_t *expert_slot);
+
+/* Looks up the n expert ids (host) one step needs in `layer`. For each id
+ * writes its slot (host slot_of_id[n]); misses are assigned a victim slot,
+ * the least recently used slot that this step does not need, and listed in
+ * miss_ids (host, capacity n). Duplicate ids count once. More distinct ids
+ * than slots -> MOE_ERR_CAPACITY. Resident caches (slots >= E) never miss
+ * and count nothing. */
+int slot_cache_lookup(moe_slot_cache *c, int layer, const int32_t *ids_host,
+                      int n, int32_t *slot_of_id_host,
+                      int32_t *miss_ids_host, int *n_miss);
+
+/* Copies the records of the missed experts from the pinned pool into their
+ * slots on `side` (one cudaMemcpyAsync each, after the layer's previous
+ * readers released it), updates the layer's device expert_slot table, and
+ * makes `compute` wait for all of it. */
+int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss_ids_host,
+                    int n_miss, moe_stream_t side, moe_stream_t compute);
+
+/* Marks the end of this step's reads of `layer`'s slots on `compute`; the
+ * next fill of the layer waits for this point before overwriting a slot. */
+int slot_cache_release(moe_slot_cache *c, int layer, moe_stream_t compute);
+
+int slot_cache_stats(const moe_slot_cache *c, uint64_t *hits,
+                     uint64_t *misses, uint64_t *h2d_bytes);
+
+/* Test hook: the next `count` fills fail with MOE_ERR_CUDA before copying
+ * (host-side fault injection; no device is touched). */
+int slot_cache_inject_fill_failure(moe_slot_cache *c, int count);
+
+void slot_cache_destroy(moe_slot_cache *c);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACTMOE_H */

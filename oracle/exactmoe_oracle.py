@@ -285,6 +285,25 @@ class PackedExperts:
         return self._cache(int(e))
 
 
+class LazyQuantizedExperts:
+    """Experts quantised by this oracle on first use, from a function that
+    returns expert e's BF16-valued (gate [I][H], up [I][H], down [H][I])."""
+
+    def __init__(self, weights_of, E: int, H: int, I: int, cache: int = 80):
+        self.weights_of, self.E, self.H, self.I = weights_of, E, H, I
+        self._cache = lru_cache(maxsize=cache)(self._deq)
+
+    def _deq(self, e: int):
+        return tuple(dequantize_packed(*quantize_pack(w)) for w in self.weights_of(e))
+
+    def packed(self, e: int):
+        """(packed, scale bits) of gate, up, down of expert e."""
+        return tuple(quantize_pack(w) for w in self.weights_of(e))
+
+    def dequantized(self, e: int):
+        return self._cache(int(e))
+
+
 def grouped_ffn(x, experts: PackedExperts, sorted_pair, offsets, k: int):
     """Grouped form: per expert, its rows in sorted order.
 

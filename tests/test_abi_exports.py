@@ -1,0 +1,165 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point include/*.h declares, and rejects bad arguments before touching CUDA.
+The slot cache's host bookkeeping (LRU, capacity, rollback on an injected
+fill failure) runs here too: lookups touch no device memory."""
+import ctypes as C
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ ]*[\s\*]+\**([a-z_][a-z0-9_]*)\s*\(", src, re.M):
+            names.append(m.group(1))
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def native():
+    from w4a16_mixture_experts_moe_b200 import build
+    build.build()
+    from w4a16_mixture_experts_moe_b200 import _native
+    return _native
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for want in ["moe_quantize_pack", "moe_route_topk", "moe_group_tokens", "moe_grouped_w4a16_ffn",
+                 "moe_combine", "slot_cache_lookup", "slot_cache_fill"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(native):
+    lib = C.CDLL(native.LIB_PATH)
+    names = _declared_functions()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(names) <= set(native.SIGNATURES), set(names) - set(native.SIGNATURES)
+
+
+def test_record_layout(native):
+    L = native.moe_expert_record_layout(2048, 1024)
+    assert L["bytes"] == 3 * 1024 * 2048 // 2 + 3 * (1024 * 2048 // 128) * 2 == 3244032
+    assert all(v % 256 == 0 for v in L.values())
+    with pytest.raises(native.MoeError) as ei:
+        native.moe_expert_record_layout(2048, 1000)
+    assert ei.value.status == 2
+
+
+def test_argument_checks_run_before_any_cuda_call(native):
+    lib = native.lib
+    assert lib.moe_quantize_pack(16, 1, 1, 100, 16, 0, 16, 0, None) == native.MOE_ERR_SHAPE
+    assert b"K=100" in lib.moe_last_error()
+    assert lib.moe_route_topk(16, 16, 4, 256, 300, 2, None, 0, 16, 16, 16, None) == native.MOE_ERR_SHAPE
+    assert lib.moe_route_topk(16, 16, 4, 256, 8, 9, None, 0, 16, 16, 16, None) == native.MOE_ERR_SHAPE
+    assert lib.moe_route_topk(16, 16, 4, 256, 8, 2, None, 64, 16, 16, 16, None) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_group_tokens(16, 4, 2, 8, 16, 16, 16, 16, 256, 1, None) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_w4a16_ffn(16, 16, 16, 256, 3244032, None, 64, 4, 8, 64, 2048, 1000, 0,
+                                     16, 256, 1 << 20, None) == native.MOE_ERR_SHAPE
+    assert lib.moe_grouped_w4a16_ffn(16, 16, 16, 256, 1000, None, 64, 4, 8, 64, 2048, 1024, 0,
+                                     16, 256, 1 << 20, None) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_w4a16_ffn(16, 16, 16, 256, 3244032, None, 64, 4, 8, 64, 2048, 1024, 7,
+                                     16, 256, 1 << 20, None) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(16, 16, 16, None, 4, 40, 2048, 16, None) == native.MOE_ERR_SHAPE
+    # T == 0 is a no-op that launches nothing
+    assert lib.moe_combine(None, None, None, None, 0, 2, 2048, None, None) == native.MOE_OK
+    assert lib.moe_route_topk(None, None, 0, 2048, 64, 8, None, 0, None, None, None, None) == native.MOE_OK
+
+
+class _LRUModel:
+    """Plain model of the slot cache policy for the host tests."""
+
+    def __init__(self, E, S):
+        self.E, self.S = E, S
+        self.owner = [-1] * S
+        self.stamp = [0] * S
+        self.where = {}
+        self.now = 0
+        self.hits = self.misses = 0
+
+    def lookup(self, ids):
+        self.now += 1
+        uniq = list(dict.fromkeys(ids))
+        miss = []
+        for e in uniq:
+            if e in self.where:
+                self.stamp[self.where[e]] = self.now
+                self.hits += 1
+            else:
+                miss.append(e)
+        for e in miss:
+            free = [s for s in range(self.S) if self.stamp[s] != self.now and self.owner[s] < 0]
+            if free:
+                v = free[0]
+            else:
+                cands = [s for s in range(self.S) if self.stamp[s] != self.now]
+                v = min(cands, key=lambda s: (self.stamp[s], s))
+            if self.owner[v] >= 0:
+                del self.where[self.owner[v]]
+            self.owner[v] = e
+            self.where[e] = v
+            self.stamp[v] = self.now
+            self.misses += 1
+        return [self.where[e] for e in ids], miss
+
+
+def test_slot_cache_lru_matches_model(native):
+    import numpy as np
+    import synth
+    E, S, k, steps = 64, 16, 8, 200
+    c = native.SlotCache(1, E, S, 256, 0x1000, 0x2000, 0x3000)   # fake addresses: lookups never dereference
+    model = _LRUModel(E, S)
+    routing = synth.drawn_routing(0, E, k, steps)
+    for s in range(steps):
+        ids = [int(v) for v in routing[s]]
+        got = c.lookup(0, ids)
+        want = model.lookup(ids)
+        assert got == want, s
+        # every id maps to a distinct slot this step
+        assert len(set(got[0])) == len(ids)
+    st = c.stats()
+    assert (st["hits"], st["misses"]) == (model.hits, model.misses)
+    assert st["h2d_bytes"] == 0      # no fill was issued
+    # keep-probability 0.5 routing over 16 slots: a fair share of hits
+    assert 0.3 < st["hits"] / (st["hits"] + st["misses"]) < 0.9
+    c.close()
+
+
+def test_slot_cache_capacity_duplicates_and_resident_mode(native):
+    c = native.SlotCache(2, 8, 2, 256, 0x1000, 0x2000, 0x3000)
+    with pytest.raises(native.MoeError) as ei:
+        c.lookup(0, [0, 1, 2])
+    assert ei.value.status == native.MOE_ERR_CAPACITY
+    slots, miss = c.lookup(1, [5, 5, 5])
+    assert len(set(slots)) == 1 and miss == [5]
+    c.close()
+    r = native.SlotCache(1, 8, 8, 256, 0x1000, 0x2000, 0x3000)
+    slots, miss = r.lookup(0, [3, 1])
+    assert slots == [3, 1] and miss == [3, 1]          # first touch loads
+    slots, miss = r.lookup(0, [3, 1, 7])
+    assert slots == [3, 1, 7] and miss == [7]
+    assert r.stats() == {"hits": 0, "misses": 0, "h2d_bytes": 0}   # accounting bypassed
+    r.close()
+
+
+def test_slot_cache_injected_fill_failure_rolls_back(native):
+    c = native.SlotCache(1, 8, 4, 256, 0x1000, 0x2000, 0x3000)
+    _, miss = c.lookup(0, [1, 2])
+    c.inject_fill_failure(1)
+    with pytest.raises(native.MoeError) as ei:
+        c.fill(0, miss, side=0, compute=0)
+    assert ei.value.status == native.MOE_ERR_CUDA and "injected" in str(ei.value)
+    # the failed experts are not resident: the next lookup misses them again
+    _, miss2 = c.lookup(0, [1, 2])
+    assert sorted(miss2) == [1, 2]
+    with pytest.raises(native.MoeError):
+        c.fill(0, [5], side=0, compute=0)                 # never assigned by a lookup
+    c.close()

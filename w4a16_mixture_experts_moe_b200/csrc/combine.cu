@@ -1,0 +1,64 @@
+// A7 — router-weighted combine of the k expert outputs of each token, with
+// an optional residual: out[t] = bf16_rn(res[t] + sum_j w[t][j] * y[pos(t,j)]),
+// fp32 accumulation in increasing j (deterministic). One CTA per token; each
+// thread owns 8 consecutive hidden elements (16-byte loads and stores).
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int CB_THREADS = 256;
+
+__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t *__restrict__ y,
+                                                              const float *__restrict__ topk_w,
+                                                              const int32_t *__restrict__ pair_pos,
+                                                              const uint16_t *residual, int k, int H,
+                                                              uint16_t *out) {
+  __shared__ float ws[MAX_K];
+  __shared__ int32_t ps[MAX_K];
+  const int t = blockIdx.x;
+  if (threadIdx.x < k) {
+    ws[threadIdx.x] = topk_w[int64_t(t) * k + threadIdx.x];
+    ps[threadIdx.x] = pair_pos[int64_t(t) * k + threadIdx.x];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < H / 8; c += CB_THREADS) {
+    float acc[8];
+    if (residual) {
+      const uint4 r = reinterpret_cast<const uint4 *>(residual + int64_t(t) * H)[c];
+      acc[0] = bf16_lo(r.x); acc[1] = bf16_hi(r.x); acc[2] = bf16_lo(r.y); acc[3] = bf16_hi(r.y);
+      acc[4] = bf16_lo(r.z); acc[5] = bf16_hi(r.z); acc[6] = bf16_lo(r.w); acc[7] = bf16_hi(r.w);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    }
+    for (int j = 0; j < k; ++j) {
+      const int pos = ps[j];
+      if (pos < 0) continue;
+      const float w = ws[j];
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + int64_t(pos) * H) + c);
+      acc[0] = fmaf(w, bf16_lo(v.x), acc[0]); acc[1] = fmaf(w, bf16_hi(v.x), acc[1]);
+      acc[2] = fmaf(w, bf16_lo(v.y), acc[2]); acc[3] = fmaf(w, bf16_hi(v.y), acc[3]);
+      acc[4] = fmaf(w, bf16_lo(v.z), acc[4]); acc[5] = fmaf(w, bf16_hi(v.z), acc[5]);
+      acc[6] = fmaf(w, bf16_lo(v.w), acc[6]); acc[7] = fmaf(w, bf16_hi(v.w), acc[7]);
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]); o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]); o.w = pack_bf16x2(acc[6], acc[7]);
+    reinterpret_cast<uint4 *>(out + int64_t(t) * H)[c] = o;
+  }
+}
+
+}  // namespace moe
+
+extern "C" int moe_combine(const moe_bf16 *y, const float *topk_w, const int32_t *pair_pos,
+                           const moe_bf16 *residual, int T, int k, int H, moe_bf16 *out, moe_stream_t stream) {
+  using namespace moe;
+  if (T < 0 || k < 1 || k > MAX_K || H < 8 || H % 8)
+    return set_error(MOE_ERR_SHAPE, "moe_combine: T=%d k=%d H=%d (need T>=0, 1<=k<=32, H a multiple of 8)", T, k, H);
+  if (T == 0) return MOE_OK;
+  if (!y || !topk_w || !pair_pos || !out) return set_error(MOE_ERR_INVALID_ARG, "moe_combine: NULL pointer");
+  if (!aligned(y, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)))
+    return set_error(MOE_ERR_INVALID_ARG, "moe_combine: y, residual and out must be 16-byte aligned");
+  combine_kernel<<<T, CB_THREADS, 0, as_stream(stream)>>>(y, topk_w, pair_pos, residual, k, H, out);
+  return check_launch("moe_combine");
+}

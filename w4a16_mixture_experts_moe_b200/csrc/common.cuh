@@ -1,0 +1,54 @@
+// Shared helpers of the CUDA library: status plumbing, BF16 bit helpers,
+// device error word. Nothing here is shared with the CPU oracle.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/exactmoe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- host side
+int set_error(int status, const char *fmt, ...);
+// Checks the launch status and adds n to the process-wide count of kernels
+// this library has enqueued.
+int check_launch(const char *what, int n = 1);
+void count_launches(int n);
+// Raises a kernel's dynamic shared-memory limit on the current device (once
+// per device and kernel; later calls are a lookup).
+int allow_dynamic_smem(const void *kernel, size_t bytes, const char *what);
+
+static inline cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+static inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int GROUP = 128;
+constexpr int MAX_E = 256;
+constexpr int MAX_K = 32;
+constexpr size_t WS_HEADER = 256;  // error word + scheduler counters
+
+// ---------------------------------------------------------------- device side
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_to_f(uint16_t v) { return __uint_as_float(uint32_t(v) << 16); }
+
+__device__ __forceinline__ uint16_t f_to_bf16(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t *>(&b);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// First writer wins; later codes are dropped.
+__device__ __forceinline__ void flag_error(int32_t *err, int32_t code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+}  // namespace moe

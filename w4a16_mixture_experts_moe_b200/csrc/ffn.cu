@@ -1,0 +1,73 @@
+// Entry point of the grouped W4A16 SwiGLU expert FFN (A5 + A6): argument
+// checks, workspace layout and the choice between the decode-sized GEMV path
+// and the prefill-sized tensor-core path.
+#include "ffn.cuh"
+
+namespace moe {
+
+static size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Average rows per expert at which the tensor-core path takes over.
+constexpr int TC_MIN_ROWS_PER_EXPERT = 32;
+
+}  // namespace moe
+
+extern "C" size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path) {
+  (void)E; (void)H; (void)path;
+  if (T < 0 || k < 1 || I < 0) return moe::WS_HEADER;
+  return moe::WS_HEADER + moe::round256(size_t(T) * size_t(k) * size_t(I) * 2);
+}
+
+extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair, const int32_t *offsets,
+                                     const void *bank, int64_t record_bytes, const int32_t *expert_slot,
+                                     int n_slots, int T, int k, int E, int H, int I, int path, moe_bf16 *y,
+                                     void *ws, size_t ws_bytes, moe_stream_t stream) {
+  using namespace moe;
+  if (T < 0 || E < 1 || E > MAX_E || k < 1 || k > E || k > MAX_K)
+    return set_error(MOE_ERR_SHAPE, "moe_grouped_w4a16_ffn: T=%d E=%d k=%d (need T>=0, 1<=E<=256, 1<=k<=min(E,32))",
+                     T, E, k);
+  if (H < GROUP || I < GROUP || H % GROUP || I % GROUP)
+    return set_error(MOE_ERR_SHAPE, "moe_grouped_w4a16_ffn: H=%d I=%d must be positive multiples of 128", H, I);
+  if (int64_t(T) * k > (int64_t(1) << 30))
+    return set_error(MOE_ERR_SHAPE, "moe_grouped_w4a16_ffn: T*k too large");
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_TC)
+    return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: unknown path %d", path);
+  moe_record_layout L;
+  int st = moe_expert_record_layout(H, I, &L);
+  if (st != MOE_OK) return st;
+  if (!offsets || !bank || !ws || (T > 0 && (!x || !sorted_pair || !y)))
+    return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: NULL pointer");
+  if (record_bytes < L.bytes || record_bytes % 256)
+    return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: record_bytes=%lld (need >= %lld, multiple of 256)",
+                     (long long)record_bytes, (long long)L.bytes);
+  if (n_slots < 1 || (!expert_slot && n_slots < E))
+    return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: n_slots=%d (identity mapping needs >= E)", n_slots);
+  if (!aligned(bank, 256) || !aligned(ws, 256) || (T > 0 && (!aligned(x, 16) || !aligned(y, 16))))
+    return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: bank/ws need 256-byte, x/y 16-byte alignment");
+  if (ws_bytes < moe_ffn_workspace_size(T, k, E, H, I, path))
+    return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: workspace %zu B < %zu B", ws_bytes,
+                     moe_ffn_workspace_size(T, k, E, H, I, path));
+
+  cudaStream_t s = as_stream(stream);
+  FfnArgs a;
+  a.x = x; a.sorted_pair = sorted_pair; a.offsets = offsets;
+  a.bank = static_cast<const uint8_t *>(bank); a.expert_slot = expert_slot;
+  a.rec = record_bytes; a.n_slots = n_slots;
+  a.T = T; a.k = k; a.E = E; a.H = H; a.I = I;
+  a.off_gq = L.gate_q; a.off_uq = L.up_q; a.off_dq = L.down_q;
+  a.off_gs = L.gate_s; a.off_us = L.up_s; a.off_ds = L.down_s;
+  a.err = static_cast<int32_t *>(ws);
+  a.h = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER);
+  a.y = y;
+  if (cudaMemsetAsync(a.err, 0, sizeof(int32_t), s) != cudaSuccess) return check_launch("moe_grouped_w4a16_ffn memset");
+  if (T == 0) return MOE_OK;
+
+  int chosen = path;
+  if (path == MOE_PATH_AUTO)
+    chosen = (int64_t(T) * k >= int64_t(TC_MIN_ROWS_PER_EXPERT) * E) ? MOE_PATH_TC : MOE_PATH_GEMV;
+  if (chosen == MOE_PATH_TC) {
+    st = launch_ffn_tc(a, s);
+    if (st != MOE_ERR_UNSUPPORTED || path == MOE_PATH_TC) return st;
+  }
+  return launch_ffn_gemv(a, s);
+}

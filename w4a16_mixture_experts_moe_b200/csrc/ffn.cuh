@@ -1,0 +1,59 @@
+// Shared declarations of the grouped W4A16 expert FFN paths.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Everything a grouped-FFN kernel needs, passed by value.
+struct FfnArgs {
+  const uint16_t *x;           // [T][H]
+  const int32_t *sorted_pair;  // [P]
+  const int32_t *offsets;      // [E+1]
+  const uint8_t *bank;         // records of `rec` bytes
+  const int32_t *expert_slot;  // [E] or nullptr (identity)
+  int64_t rec;
+  int n_slots;
+  int T, k, E, H, I;
+  int64_t off_gq, off_uq, off_dq, off_gs, off_us, off_ds;  // record layout
+  uint16_t *h;    // [P][I] workspace, sorted order
+  uint16_t *y;    // [P][H] output, sorted order
+  int32_t *err;   // device error word
+};
+
+// Record of expert e, or nullptr (and the error flagged) if it has no slot.
+__device__ __forceinline__ const uint8_t *expert_record(const FfnArgs &a, int e) {
+  const int slot = a.expert_slot ? a.expert_slot[e] : e;
+  if (slot < 0 || slot >= a.n_slots) {
+    flag_error(a.err, MOE_DEVERR_NOT_RESIDENT);
+    return nullptr;
+  }
+  return a.bank + int64_t(slot) * a.rec;
+}
+
+// Offset-binary nibbles of one packed word -> four BF16x2 code pairs
+// (q_{2i}, q_{2i+1}), exact small integers: OR-ing a nibble into the
+// mantissa of BF16 128.0 gives 128 + u; subtracting 136 gives u - 8.
+__device__ __forceinline__ void dequant_codes(uint32_t w, uint32_t (&q)[4]) {
+  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t t = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+    __nv_bfloat162 v = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&t), bias);
+    q[i] = *reinterpret_cast<uint32_t *>(&v);
+  }
+}
+
+// Streaming 16-byte load that skips L1 (weights are read once).
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s);
+int launch_ffn_tc(const FfnArgs &a, cudaStream_t s);
+
+}  // namespace moe

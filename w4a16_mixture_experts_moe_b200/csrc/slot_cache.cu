@@ -1,0 +1,250 @@
+// A8 — GPU-resident expert slot cache over a pinned host pool (ExactMoE
+// paper, Abstract: a configurable GPU-resident slot cache over experts kept in
+// pinned host memory; Figure 1 caption: the pinned pool keeps every packed
+// expert and a miss transfers packed weights and scales; Figure 2 caption:
+// at full capacity every expert is resident and lookup accounting is
+// bypassed; Table 1: slot counts 8/16/32/64 with hit rate and H2D traffic).
+//
+// Host side: one LRU per layer over `slots` device records. A miss evicts the
+// least recently used slot that the current step does not need and is filled
+// with one cudaMemcpyAsync of the expert's whole record (packed codes and
+// scales, no dequantised copy) on a side stream. The layer's device table
+// expert -> slot is rewritten by a one-block kernel whose argument carries the
+// whole table, so no host buffer has to outlive the call.
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "common.cuh"
+
+namespace moe {
+
+struct SlotTable {
+  int32_t slot_of[MAX_E];
+};
+
+__global__ void write_slot_table_kernel(int32_t *dst, int E, const SlotTable table) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) dst[e] = table.slot_of[e];
+}
+
+}  // namespace moe
+
+struct moe_slot_cache {
+  int layers, E, slots;
+  int64_t rec;
+  const uint8_t *pool;
+  uint8_t *dev_slots;
+  int32_t *dev_table;
+  bool resident;
+  // per layer
+  std::vector<std::vector<int32_t>> owner;     // [layer][slot] expert or -1
+  std::vector<std::vector<int32_t>> where;     // [layer][expert] slot or -1
+  std::vector<std::vector<uint8_t>> loaded;    // [layer][expert] (resident mode)
+  std::vector<std::vector<uint64_t>> stamp;    // [layer][slot] last step that used it
+  std::vector<uint64_t> step;                  // [layer]
+  std::vector<cudaEvent_t> released, filled;   // [layer], created on first use
+  std::vector<bool> release_recorded;
+  // misses of the last lookup per layer, for rollback if the fill fails
+  std::vector<std::vector<int32_t>> pending_ids, pending_slots;
+  uint64_t hits = 0, misses = 0, h2d_bytes = 0;
+  int inject_fail = 0;
+};
+
+extern "C" int slot_cache_create(moe_slot_cache **out, int layers, int E, int slots, int64_t record_bytes,
+                                 const void *pinned_pool, void *device_slots, int32_t *expert_slot) {
+  using namespace moe;
+  if (!out) return set_error(MOE_ERR_INVALID_ARG, "slot_cache_create: out is NULL");
+  *out = nullptr;
+  if (layers < 1 || E < 1 || E > MAX_E || slots < 1 || record_bytes < 256 || record_bytes % 256)
+    return set_error(MOE_ERR_SHAPE, "slot_cache_create: layers=%d E=%d slots=%d record_bytes=%lld", layers, E, slots,
+                     (long long)record_bytes);
+  if (!pinned_pool || !device_slots || !expert_slot)
+    return set_error(MOE_ERR_INVALID_ARG, "slot_cache_create: NULL pointer");
+  moe_slot_cache *c = new moe_slot_cache();
+  c->layers = layers; c->E = E; c->slots = slots; c->rec = record_bytes;
+  c->pool = static_cast<const uint8_t *>(pinned_pool);
+  c->dev_slots = static_cast<uint8_t *>(device_slots);
+  c->dev_table = expert_slot;
+  c->resident = slots >= E;
+  c->owner.assign(layers, std::vector<int32_t>(slots, -1));
+  c->where.assign(layers, std::vector<int32_t>(E, -1));
+  c->loaded.assign(layers, std::vector<uint8_t>(E, 0));
+  c->stamp.assign(layers, std::vector<uint64_t>(slots, 0));
+  c->step.assign(layers, 0);
+  c->released.assign(layers, nullptr);
+  c->filled.assign(layers, nullptr);
+  c->release_recorded.assign(layers, false);
+  c->pending_ids.assign(layers, {});
+  c->pending_slots.assign(layers, {});
+  if (c->resident) {
+    for (int l = 0; l < layers; ++l)
+      for (int e = 0; e < E; ++e) { c->owner[l][e] = e; c->where[l][e] = e; }
+  }
+  *out = c;
+  return MOE_OK;
+}
+
+extern "C" int slot_cache_lookup(moe_slot_cache *c, int layer, const int32_t *ids, int n, int32_t *slot_of_id,
+                                 int32_t *miss_ids, int *n_miss) {
+  using namespace moe;
+  if (!c || !n_miss || (n > 0 && (!ids || !slot_of_id || !miss_ids)))
+    return set_error(MOE_ERR_INVALID_ARG, "slot_cache_lookup: NULL pointer");
+  if (layer < 0 || layer >= c->layers || n < 0)
+    return set_error(MOE_ERR_INVALID_ARG, "slot_cache_lookup: layer=%d n=%d", layer, n);
+  *n_miss = 0;
+  for (int i = 0; i < n; ++i)
+    if (ids[i] < 0 || ids[i] >= c->E) return set_error(MOE_ERR_INVALID_ARG, "slot_cache_lookup: id %d out of range", ids[i]);
+  auto &owner = c->owner[layer];
+  auto &where = c->where[layer];
+  auto &stamp = c->stamp[layer];
+  c->pending_ids[layer].clear();
+  c->pending_slots[layer].clear();
+  const uint64_t now = ++c->step[layer];
+
+  // distinct ids, first occurrence order
+  std::vector<int32_t> uniq;
+  std::vector<uint8_t> seen(c->E, 0);
+  for (int i = 0; i < n; ++i)
+    if (!seen[ids[i]]) { seen[ids[i]] = 1; uniq.push_back(ids[i]); }
+  if (int(uniq.size()) > c->slots)
+    return set_error(MOE_ERR_CAPACITY, "slot_cache_lookup: %d distinct experts > %d slots", int(uniq.size()), c->slots);
+
+  if (c->resident) {  // every expert owns its slot; only first touches load
+    for (int32_t e : uniq)
+      if (!c->loaded[layer][e]) {
+        miss_ids[(*n_miss)++] = e;
+        c->pending_ids[layer].push_back(e);
+        c->pending_slots[layer].push_back(e);
+        c->loaded[layer][e] = 1;
+      }
+    for (int i = 0; i < n; ++i) slot_of_id[i] = ids[i];
+    return MOE_OK;
+  }
+
+  // hits first, so their slots are protected from eviction this step
+  std::vector<int32_t> missing;
+  for (int32_t e : uniq) {
+    if (where[e] >= 0) { stamp[where[e]] = now; ++c->hits; }
+    else missing.push_back(e);
+  }
+  for (int32_t e : missing) {
+    int victim = -1;
+    for (int s = 0; s < c->slots; ++s) {  // a free slot, else the least recently used
+      if (stamp[s] == now) continue;
+      if (owner[s] < 0) { victim = s; break; }
+      if (victim < 0 || stamp[s] < stamp[victim]) victim = s;
+    }
+    if (victim < 0) return set_error(MOE_ERR_CAPACITY, "slot_cache_lookup: no evictable slot");
+    if (owner[victim] >= 0) where[owner[victim]] = -1;
+    owner[victim] = e;
+    where[e] = victim;
+    stamp[victim] = now;
+    ++c->misses;
+    miss_ids[(*n_miss)++] = e;
+    c->pending_ids[layer].push_back(e);
+    c->pending_slots[layer].push_back(victim);
+  }
+  for (int i = 0; i < n; ++i) slot_of_id[i] = where[ids[i]];
+  return MOE_OK;
+}
+
+static int ensure_events(moe_slot_cache *c, int layer) {
+  using namespace moe;
+  if (!c->filled[layer]) {
+    cudaError_t e = cudaEventCreateWithFlags(&c->filled[layer], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->released[layer], cudaEventDisableTiming);
+    if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "slot_cache: event creation: %s", cudaGetErrorString(e));
+  }
+  return MOE_OK;
+}
+
+static void rollback(moe_slot_cache *c, int layer) {
+  auto &ids = c->pending_ids[layer];
+  auto &sl = c->pending_slots[layer];
+  for (size_t i = 0; i < ids.size(); ++i) {
+    if (c->resident) { c->loaded[layer][ids[i]] = 0; continue; }
+    c->where[layer][ids[i]] = -1;
+    c->owner[layer][sl[i]] = -1;
+  }
+  ids.clear();
+  sl.clear();
+}
+
+extern "C" int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss_ids, int n_miss, moe_stream_t side,
+                               moe_stream_t compute) {
+  using namespace moe;
+  if (!c || (n_miss > 0 && !miss_ids)) return set_error(MOE_ERR_INVALID_ARG, "slot_cache_fill: NULL pointer");
+  if (layer < 0 || layer >= c->layers || n_miss < 0)
+    return set_error(MOE_ERR_INVALID_ARG, "slot_cache_fill: layer=%d n_miss=%d", layer, n_miss);
+  if (n_miss == 0) return MOE_OK;
+  for (int i = 0; i < n_miss; ++i)
+    if (miss_ids[i] < 0 || miss_ids[i] >= c->E || c->where[layer][miss_ids[i]] < 0)
+      return set_error(MOE_ERR_INVALID_ARG, "slot_cache_fill: id %d was not assigned a slot by slot_cache_lookup",
+                       miss_ids[i]);
+  if (c->inject_fail > 0) {
+    --c->inject_fail;
+    rollback(c, layer);
+    return set_error(MOE_ERR_CUDA, "slot_cache_fill: injected fill failure (layer %d)", layer);
+  }
+  int st = ensure_events(c, layer);
+  if (st != MOE_OK) { rollback(c, layer); return st; }
+  cudaStream_t s = as_stream(side), cs = as_stream(compute);
+  cudaError_t e = cudaSuccess;
+  if (c->release_recorded[layer]) e = cudaStreamWaitEvent(s, c->released[layer], 0);
+  for (int i = 0; i < n_miss && e == cudaSuccess; ++i) {
+    const int id = miss_ids[i];
+    const int slot = c->where[layer][id];
+    uint8_t *dst = c->dev_slots + (int64_t(layer) * c->slots + slot) * c->rec;
+    const uint8_t *src = c->pool + (int64_t(layer) * c->E + id) * c->rec;
+    e = cudaMemcpyAsync(dst, src, size_t(c->rec), cudaMemcpyHostToDevice, s);
+  }
+  if (e != cudaSuccess) {
+    rollback(c, layer);
+    return set_error(MOE_ERR_CUDA, "slot_cache_fill: copy: %s", cudaGetErrorString(e));
+  }
+  SlotTable table;
+  for (int x = 0; x < c->E; ++x) table.slot_of[x] = c->where[layer][x];
+  write_slot_table_kernel<<<1, 256, 0, s>>>(c->dev_table + int64_t(layer) * c->E, c->E, table);
+  count_launches(1);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaEventRecord(c->filled[layer], s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, c->filled[layer], 0);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "slot_cache_fill: %s", cudaGetErrorString(e));
+  c->h2d_bytes += uint64_t(n_miss) * uint64_t(c->rec);
+  c->pending_ids[layer].clear();
+  c->pending_slots[layer].clear();
+  return MOE_OK;
+}
+
+extern "C" int slot_cache_release(moe_slot_cache *c, int layer, moe_stream_t compute) {
+  using namespace moe;
+  if (!c || layer < 0 || layer >= c->layers) return set_error(MOE_ERR_INVALID_ARG, "slot_cache_release: bad argument");
+  int st = ensure_events(c, layer);
+  if (st != MOE_OK) return st;
+  cudaError_t e = cudaEventRecord(c->released[layer], as_stream(compute));
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "slot_cache_release: %s", cudaGetErrorString(e));
+  c->release_recorded[layer] = true;
+  return MOE_OK;
+}
+
+extern "C" int slot_cache_stats(const moe_slot_cache *c, uint64_t *hits, uint64_t *misses, uint64_t *h2d_bytes) {
+  if (!c) return moe::set_error(MOE_ERR_INVALID_ARG, "slot_cache_stats: NULL cache");
+  if (hits) *hits = c->hits;
+  if (misses) *misses = c->misses;
+  if (h2d_bytes) *h2d_bytes = c->h2d_bytes;
+  return MOE_OK;
+}
+
+extern "C" int slot_cache_inject_fill_failure(moe_slot_cache *c, int count) {
+  if (!c || count < 0) return moe::set_error(MOE_ERR_INVALID_ARG, "slot_cache_inject_fill_failure: bad argument");
+  c->inject_fail = count;
+  return MOE_OK;
+}
+
+extern "C" void slot_cache_destroy(moe_slot_cache *c) {
+  if (!c) return;
+  for (cudaEvent_t ev : c->filled) if (ev) cudaEventDestroy(ev);
+  for (cudaEvent_t ev : c->released) if (ev) cudaEventDestroy(ev);
+  delete c;
+}
