@@ -34,9 +34,9 @@ notes of the repository):
 * grouping: per-expert counts, exclusive prefix sum, and the stable
   permutation of flat pair indices p = t*k + j by expert;
 * expert FFN (SwiGLU): g = x Wg^T, u = x Wu^T, h = bf16_rn(silu(g) * u),
-  y = bf16_rn(h Wd^T), where W = q * s dequantised exactly, sums in fp64;
-  h and y are BF16 because the experts are W4A16 (Abstract): every
-  activation an expert produces, its intermediate and its output, is BF16;
+  y = h Wd^T, where W = q * s dequantised exactly, sums in fp64; h is the
+  expert's BF16 activation (A16), y is the expert's unrounded output that the
+  combine weights (the pages do not store it, so it is not rounded);
 * combine: out_t = bf16_rn(residual_t + sum_j w_tj * y_(t,j)) in j order.
 
 Arithmetic is fp64 except where floating point decides an integer (the
@@ -250,13 +250,13 @@ def silu(g):
 def swiglu_expert(xr, wg, wu, wd):
     """Rows xr [R][H] through one expert; W already dequantised (float64).
 
-    Returns h [R][I] and y [R][H], both BF16-rounded (A16 activations).
+    Returns h [R][I] (BF16-rounded) and y [R][H] (float64).
     """
     xr = np.asarray(xr, dtype=np.float64)
     g = xr @ wg.T
     u = xr @ wu.T
     h = round_to_bf16(silu(g) * u)
-    return h, round_to_bf16(h @ wd.T)
+    return h, h @ wd.T
 
 
 class PackedExperts:
@@ -309,7 +309,7 @@ class LazyQuantizedExperts:
 def grouped_ffn(x, experts: PackedExperts, sorted_pair, offsets, k: int):
     """Grouped form: per expert, its rows in sorted order.
 
-    Returns h [T*k][I] and y [T*k][H] in sorted order (BF16 values).
+    Returns h [T*k][I] (BF16 values) and y [T*k][H] (float64) in sorted order.
     """
     x = np.asarray(x, dtype=np.float64)
     E = len(offsets) - 1
@@ -364,7 +364,7 @@ def moe_layer_per_token(x, experts: PackedExperts, ids, w, residual=None):
             g = wg.dot(x[t])
             u = wu.dot(x[t])
             h = round_to_bf16(silu(g) * u)
-            acc = acc + w[t, j] * round_to_bf16(wd.dot(h))
+            acc = acc + w[t, j] * wd.dot(h)
         out[t] = round_to_bf16(acc)
     return out
 

@@ -225,8 +225,7 @@ def test_single_expert_top1_equals_dense_swiglu():
     xt = torch.from_numpy(x)
     F = torch.nn.functional
     h = (F.silu(F.linear(xt, wg)) * F.linear(xt, wu)).to(torch.bfloat16).double()
-    y = F.linear(h, wd).to(torch.bfloat16).double()
-    ref = (torch.from_numpy(res) + y).to(torch.bfloat16).double().numpy()
+    ref = (torch.from_numpy(res) + F.linear(h, wd)).to(torch.bfloat16).double().numpy()
     assert np.array_equal(out, ref)
 
 
