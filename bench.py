@@ -36,7 +36,12 @@ sys.path.insert(0, ROOT)
 H, I, E, K, LAYERS = 2048, 1024, 64, 8, 16
 SWEEP_T = (1, 4, 16, 64)
 METRIC = "MoE-layer tokens/s; HBM GB/s (decode) and TC TFLOP/s (prefill) vs B200 peak"
-REC_BYTES = 3 * I * H // 2 + 3 * (I * H // 128) * 2   # one packed expert record
+SHAPES = {"olmoe": (2048, 1024, 64, 8), "wide": (4096, 14336, 8, 2)}   # (H, I, E, k)
+
+
+def rec_bytes(h, i):
+    """Bytes of one packed expert record: codes of three matrices + their scales."""
+    return 3 * i * h // 2 + 3 * (i * h // 128) * 2
 
 
 def parse():
@@ -50,7 +55,17 @@ def parse():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc"])
-    return ap.parse_args()
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "slotcache"],
+                    help="decode: the 16-layer stack sweep (default); prefill: one layer at large T; "
+                         "slotcache: 16 layers decoding from a pinned host pool through S GPU slots per layer")
+    ap.add_argument("--slots", type=int, default=16)
+    ap.add_argument("--shape", default="olmoe", choices=list(SHAPES))
+    a = ap.parse_args()
+    if a.workload == "prefill" and a.T == 16:
+        a.T = 8192
+    if a.workload == "prefill" and a.layers == LAYERS:
+        a.layers = 1
+    return a
 
 
 def peaks():
@@ -158,13 +173,16 @@ class Stack:
     """16 OLMoE-shaped layers: per layer a packed expert bank and a router, plus
     per-T buffers. Weights are drawn on the device with the seeded recipe."""
 
-    def __init__(self, layers, path):
+    def __init__(self, layers, path, shape="olmoe", renorm=False):
         import torch
 
         import synth
         import w4a16_mixture_experts_moe_b200 as M
         from w4a16_mixture_experts_moe_b200.layer import ExpertBank
         self.M, self.torch, self.layers = M, torch, layers
+        H, I, E, K = SHAPES[shape]
+        self.H, self.I, self.E, self.K = H, I, E, K
+        self.flags = M.MOE_RENORM if renorm else 0
         self.path = {"auto": M.MOE_PATH_AUTO, "gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC}[path]
         self.banks, self.routers = [], []
         for l in range(layers):
@@ -179,6 +197,7 @@ class Stack:
     def buffers(self, T):
         from w4a16_mixture_experts_moe_b200.layer import LayerBuffers
         torch = self.torch
+        H, I, E, K = self.H, self.I, self.E, self.K
         bufs = [LayerBuffers(T, K, E, H, I, path=self.path) for _ in range(self.layers)]
         xs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
         return bufs, xs
@@ -188,15 +207,17 @@ class Stack:
         list of (start, end) CUDA events recorded around each layer's FFN call."""
         from w4a16_mixture_experts_moe_b200.layer import moe_layer_forward
         M = self.M
+        H, I, E, K = self.H, self.I, self.E, self.K
         cur = x_in
         for l in range(self.layers):
             out = xs[l % 2] if cur is not xs[l % 2] else xs[(l + 1) % 2]
             b = bufs[l]
             T = b.T
             if events is None:
-                moe_layer_forward(cur, self.routers[l], self.banks[l], b, residual=cur, out=out)
+                moe_layer_forward(cur, self.routers[l], self.banks[l], b, flags=self.flags, residual=cur, out=out)
             else:
-                M.moe_route_topk(cur, self.routers[l], T, H, E, K, None, 0, b.logits, b.topk_ids, b.topk_w)
+                M.moe_route_topk(cur, self.routers[l], T, H, E, K, None, self.flags, b.logits, b.topk_ids,
+                                 b.topk_w)
                 M.moe_group_tokens(b.topk_ids, T, K, E, b.counts, b.offsets, b.sorted_pair, b.pair_pos,
                                    b.group_ws, b.group_ws_bytes)
                 events[l][0].record()
@@ -225,6 +246,7 @@ def measure_T(stack, T, steps, warmup, world, want_e2e=True, want_roofline=True)
     """Device-timed step, e2e step and per-call FFN timing at T tokens."""
     import synth
     torch, M = stack.torch, stack.M
+    H = stack.H
     bufs, xs = stack.buffers(T)
     x_dev = synth.activations(T, H, device="cuda")
     x_host = synth.activations(T, H).pin_memory()
@@ -272,7 +294,8 @@ def measure_T(stack, T, steps, warmup, world, want_e2e=True, want_roofline=True)
         n_act = [int((b.counts > 0).sum().item()) for b in bufs]
         res["ffn_ms_per_call"] = statistics.mean(per_call)
         res["n_active_mean"] = statistics.mean(n_act)
-        res["ffn_bytes_per_call"] = statistics.mean(n_act) * REC_BYTES
+        res["ffn_bytes_per_call"] = statistics.mean(n_act) * rec_bytes(stack.H, stack.I)
+        res["ffn_flops_per_call"] = 6.0 * T * stack.K * stack.H * stack.I
     del g, g2
     return res
 
@@ -335,6 +358,10 @@ def main():
     import torch
     rank, world, local = dist_setup(a.gpus)
     P = peaks()
+    if a.workload == "prefill":
+        return main_prefill(a, rank, world, P)
+    if a.workload == "slotcache":
+        return main_slotcache(a, rank, world, P)
     stack = Stack(a.layers, a.path)
     head = measure_T(stack, a.T, a.steps, a.warmup, world)
     sweep = {}
@@ -379,6 +406,143 @@ def main():
             "gpu_launches": head["launches_per_step"] * a.steps,
             "clocks": head["clocks"],
             "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main_slotcache(a, rank, world, P):
+    """Decode at T=1 with every expert in pinned host memory and `slots` GPU
+    slots per layer; routing drawn so each expert of the previous step is kept
+    with probability 0.5. Each step: per layer, route (weights of the drawn
+    ids), host LRU lookup, H2D fill of the misses on a side stream, group,
+    FFN through the slot table, combine."""
+    import torch
+
+    import synth
+    M = __import__("w4a16_mixture_experts_moe_b200")
+    from w4a16_mixture_experts_moe_b200.layer import LayerBuffers
+    L, S, T = a.layers, a.slots, 1
+    steps = a.steps if a.steps >= 16 else 128
+    stack = Stack(L, "auto")
+    rec = stack.banks[0].rec
+    pool = torch.empty(L * E * rec, dtype=torch.uint8, pin_memory=True)
+    for l in range(L):
+        pool[l * E * rec:(l + 1) * E * rec].copy_(stack.banks[l].buf)
+    stack.banks = None                       # the experts now live only in the pinned pool
+    torch.cuda.empty_cache()
+    slots = torch.empty(L * S * rec, dtype=torch.uint8, device="cuda")
+    table = torch.full((L, E), -1, dtype=torch.int32, device="cuda")
+    cache = M.SlotCache(L, E, S, rec, pool, slots, table)
+    routing = [synth.drawn_routing(l, E, K, a.warmup + steps) for l in range(L)]
+    ids_dev = torch.tensor([[routing[l][s] for l in range(L)] for s in range(a.warmup + steps)], dtype=torch.int32,
+                           device="cuda")
+    x0 = synth.activations(a.warmup + steps, H, device="cuda")
+    bufs = [LayerBuffers(T, K, E, H, I) for _ in range(L)]
+    xs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    side = torch.cuda.Stream()
+    comp = torch.cuda.current_stream()
+
+    # pinned host -> device copy bandwidth, same run, same size as a miss
+    probe_n = 64
+    dst = torch.empty(probe_n * rec, dtype=torch.uint8, device="cuda")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        ev0.record(side)
+        for i in range(probe_n):
+            dst[i * rec:(i + 1) * rec].copy_(pool[i * rec:(i + 1) * rec], non_blocking=True)
+        ev1.record(side)
+        side.synchronize()
+    pinned_gbs = probe_n * rec / (ev0.elapsed_time(ev1) / 1e3) / 1e9
+    del dst
+
+    def step(si):
+        cur = x0[si:si + 1]
+        for l in range(L):
+            b = bufs[l]
+            ids = [int(v) for v in routing[l][si]]
+            _, miss = cache.lookup(l, ids)
+            cache.fill(l, miss, side=side, compute=comp)
+            b.topk_ids.copy_(ids_dev[si, l:l + 1])
+            M.moe_route_topk(cur, stack.routers[l], T, H, E, K, None, M.MOE_IDS_GIVEN, b.logits, b.topk_ids,
+                             b.topk_w)
+            M.moe_group_tokens(b.topk_ids, T, K, E, b.counts, b.offsets, b.sorted_pair, b.pair_pos, b.group_ws,
+                               b.group_ws_bytes)
+            M.moe_grouped_w4a16_ffn(cur, b.sorted_pair, b.offsets, slots.data_ptr() + l * S * rec, rec, table[l], S,
+                                    T, K, E, H, I, M.MOE_PATH_AUTO, b.y, b.ffn_ws, b.ffn_ws_bytes)
+            out = xs[l % 2]
+            M.moe_combine(b.y, b.topk_w, b.pair_pos, cur, T, K, H, out)
+            cache.release(l, comp)
+            cur = out
+        return cur
+
+    for si in range(a.warmup):
+        step(si)
+    torch.cuda.synchronize()
+    st0 = cache.stats()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = M.moe_launch_counter()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        s0.record()
+        for si in range(a.warmup, a.warmup + steps):
+            step(si)
+        s1.record()
+        torch.cuda.synchronize()
+    launches = M.moe_launch_counter() - launches0
+    ms = s0.elapsed_time(s1) / steps
+    st1 = cache.stats()
+    hits, misses = st1["hits"] - st0["hits"], st1["misses"] - st0["misses"]
+    h2d = st1["h2d_bytes"] - st0["h2d_bytes"]
+    err = [M.moe_read_device_error(b.ffn_ws) for b in bufs]
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": T * L / (ms / 1e3), "unit": "layer-tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"olmoe-{L}L-slotcache-decode", "T": T, "layers": L, "slots_per_layer": S,
+                       "H": H, "I": I, "E": E, "k": K, "routing": "drawn, keep-probability 0.5",
+                       "pool": f"{L * E * rec / 1e9:.2f} GB pinned host", "parallelism": f"replicas{world}"},
+            "decode_tokens_per_s": 1e3 / ms,
+            "hit_rate": hits / max(1, hits + misses),
+            "h2d_gb": h2d / 1e9, "h2d_gb_per_step": h2d / 1e9 / steps,
+            "h2d_achieved_gbs": h2d / (ms * steps / 1e3) / 1e9, "pinned_copy_gbs": pinned_gbs,
+            "device_errors": sorted(set(err)),
+            "gpu_launches": launches, "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    cache.close()
+
+
+def main_prefill(a, rank, world, P):
+    """One layer at large T (tensor-core path); roofline = FLOPs / FFN time."""
+    H_, I_, E_, K_ = SHAPES[a.shape]
+    stack = Stack(a.layers, a.path, a.shape, renorm=(a.shape == "wide"))
+    r = measure_T(stack, a.T, a.steps, a.warmup, world)
+    if rank == 0:
+        T, L = a.T, a.layers
+        achieved = r["ffn_flops_per_call"] / (r["ffn_ms_per_call"] / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": T * L * world / (r["ms_per_step"] / 1e3), "unit": "layer-tokens/s",
+            "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": r["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{a.shape}-prefill", "T": T, "layers": L, "H": H_, "I": I_, "E": E_, "k": K_,
+                       "weights": "int4 group-128 symmetric, all experts resident",
+                       "l2": f"inputs larger than L2 ({E_ * rec_bytes(H_, I_) / 1e6:.0f} MB of packed experts)",
+                       "parallelism": f"replicas{world}"},
+            "e2e": {"value": T * L * world / (r["ms_e2e"] / 1e3), "unit": "layer-tokens/s",
+                    "h2d_bytes_per_step": T * H_ * 2, "d2h_bytes_per_step": T * H_ * 2},
+            "roofline": {"bound": "tensor", "kernel": "moe_grouped_w4a16_ffn (tcgen05 gate/up + down), per call",
+                         "achieved": achieved, "peak": P["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / P["bf16_tflops"],
+                         "frac_of_sustained": achieved / P["bf16_tflops_sustained"], "traffic": None,
+                         "peak_source": P["source"], "flops_per_call": r["ffn_flops_per_call"],
+                         "ms_per_call": r["ffn_ms_per_call"], "n_active_mean": r["n_active_mean"]},
+            "cpu_baseline": None,
+            "gpu_launches": r["launches_per_step"] * a.steps,
+            "clocks": r["clocks"],
         }
         print(json.dumps(line), flush=True)
     if world > 1:

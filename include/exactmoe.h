@@ -70,7 +70,9 @@ enum {
   MOE_DEVERR_NONE = 0,
   MOE_DEVERR_EXPERT_ID = 1,   /* a top-k id outside [0, E) */
   MOE_DEVERR_NOT_RESIDENT = 2,/* an active expert has no valid slot */
-  MOE_DEVERR_TIMEOUT = 3      /* a bounded pipeline wait ran out */
+  MOE_DEVERR_TIMEOUT = 3,     /* a bounded pipeline wait ran out */
+  MOE_DEVERR_RANGE = 4        /* an activation outside FP16 range on the
+                                 tensor-core path (|x| > 65504) */
 };
 
 /* Message for the last failed call on this host thread ("" if none). */
@@ -171,7 +173,7 @@ int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E,
  * For sorted row r of expert e (offsets[e] <= r < offsets[e+1]) and token
  * t = sorted_pair[r] / k:
  *   h[r] = bf16_rn(silu(x[t] Wg_e^T) * (x[t] Wu_e^T))      (fp32 sums)
- *   y[r] = bf16_rn(h[r] Wd_e^T)                             (fp32 sums)
+ *   y[r] = h[r] Wd_e^T                                      (fp32 sums, fp32)
  *   x            [T][H] BF16.
  *   bank         device array of expert records with stride record_bytes
  *                (moe_expert_record_layout(H, I).bytes or larger, multiple
@@ -180,29 +182,33 @@ int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E,
  *                for the identity (record e holds expert e). An active
  *                expert whose slot is outside [0, n_slots) is skipped and
  *                flagged (MOE_DEVERR_NOT_RESIDENT).
- *   y            [T*k][H] BF16, rows in sorted order.
+ *   y            [T*k][H] fp32, rows in sorted order (the expert outputs
+ *                are kept unrounded until the combine).
  *   ws           at least moe_ffn_workspace_size(T, k, E, H, I, path) bytes,
  *                256-byte aligned; holds the error word and h.
- * The GEMV path applies each group's scale to the fp32 partial sum of q*x
- * over that group; the tensor-core path dequantises q*s to BF16 (one
- * rounding) before the MMA.
+ * Both paths form exact products x*(q*s) and sum them in fp32: the GEMV path
+ * applies each group's scale to the fp32 partial sum of q*x over that group;
+ * the tensor-core path dequantises q*s to FP16 (exact: at most 11 significant
+ * bits) and feeds FP16 copies of the activations (exact for BF16 values up
+ * to 65504 in magnitude; larger ones are flagged MOE_DEVERR_RANGE).
  */
 size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path);
 int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair,
                           const int32_t *offsets, const void *bank,
                           int64_t record_bytes, const int32_t *expert_slot,
                           int n_slots, int T, int k, int E, int H, int I,
-                          int path, moe_bf16 *y, void *ws, size_t ws_bytes,
+                          int path, float *y, void *ws, size_t ws_bytes,
                           moe_stream_t stream);
 
 /*
  * A7 — router-weighted combine (implied by the MoE layer; the pages do not
  * spell it out):
  *   out[t] = bf16_rn(residual[t] + sum_{j=0..k-1} topk_w[t][j] * y[pair_pos[t*k+j]])
- * summed in fp32 in increasing j. residual may be NULL (zero); pairs with
- * pair_pos < 0 contribute nothing. out may alias residual.
+ * with y the fp32 expert outputs [T*k][H], summed in fp32 in increasing j.
+ * residual may be NULL (zero); pairs with pair_pos < 0 contribute nothing.
+ * out may alias residual.
  */
-int moe_combine(const moe_bf16 *y, const float *topk_w,
+int moe_combine(const float *y, const float *topk_w,
                 const int32_t *pair_pos, const moe_bf16 *residual,
                 int T, int k, int H, moe_bf16 *out, moe_stream_t stream);
 

@@ -155,6 +155,7 @@ def test_group_tokens_bitexact(M, T, k, E, skew):
     rng = np.random.default_rng(T * 31 + k)
     if skew:
         p = np.exp(synth.zipf_log_bias(E).astype(np.float64))
+        p = p / p.sum()
         ids = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)])
     else:
         ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]) if T else np.zeros((0, k))
@@ -195,15 +196,16 @@ def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None):
     pp = torch.empty(T * k, dtype=torch.int32, device="cuda")
     gws = torch.empty(M.moe_group_workspace_size(T, k, E), dtype=torch.uint8, device="cuda")
     M.moe_group_tokens(d, T, k, E, counts, offsets, sp, pp, gws, gws.numel())
-    y = torch.full((T * k, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y = torch.full((T * k, H), float("nan"), dtype=torch.float32, device="cuda")
     nb = M.moe_ffn_workspace_size(T, k, E, H, I, path)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     es = None if expert_slot is None else torch.tensor(expert_slot, dtype=torch.int32, device="cuda")
     M.moe_grouped_w4a16_ffn(x.cuda(), sp, offsets, bank.ptr, bank.rec, es, bank.n if n_slots is None else n_slots,
                             T, k, E, H, I, path, y, ws, nb)
     code = M.moe_read_device_error(ws)
-    h = ws[256:256 + T * k * I * 2].view(torch.bfloat16).view(T * k, I)
-    return bf16_np(y), bf16_np(h), code
+    # h is internal: BF16 on the GEMV path, the BF16-rounded value held in FP16 on the tensor-core path
+    h = ws[256:256 + T * k * I * 2].view(torch.float16 if path == M.MOE_PATH_TC else torch.bfloat16).view(T * k, I)
+    return y.cpu().double().numpy(), h.float().cpu().double().numpy(), code
 
 
 @pytest.mark.parametrize("path", ["gemv", "tc"])
@@ -244,7 +246,7 @@ def test_grouped_ffn_not_resident_is_flagged(M):
 @pytest.mark.parametrize("T,k,H,res", [(16, 8, 2048, True), (5, 2, 4096, False), (1, 8, 2048, True)])
 def test_combine(M, T, k, H, res):
     rng = np.random.default_rng(T + k)
-    y = synth.normal_bf16((T * k, H), 0.5, 77)
+    y = synth.normal_bf16((T * k, H), 0.5, 77).float() * 1.001   # fp32 values with low bits set
     w = torch.from_numpy(rng.random((T, k)).astype(np.float32))
     pp = torch.from_numpy(rng.permutation(T * k).astype(np.int32))
     r = synth.activations(T, H, seed=78) if res else None
@@ -252,5 +254,6 @@ def test_combine(M, T, k, H, res):
     M.moe_combine(y.cuda(), w.cuda(), pp.cuda(), None if r is None else r.cuda(), T, k, H, out)
     torch.cuda.synchronize()
     ref = o.combine(y.double().numpy(), w.double().numpy(), pp.numpy(), None if r is None else r.double().numpy())
+    assert y.dtype == torch.float32
     assert_bf16_close(bf16_np(out), ref, "combine")
     assert np.mean(bf16_np(out) == ref) > 0.99   # one final rounding on both sides

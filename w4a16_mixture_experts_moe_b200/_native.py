@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 lib = C.CDLL(LIB_PATH)
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_CUDA, MOE_ERR_CAPACITY, MOE_ERR_DEVICE, MOE_ERR_UNSUPPORTED = range(7)
-MOE_DEVERR_NONE, MOE_DEVERR_EXPERT_ID, MOE_DEVERR_NOT_RESIDENT, MOE_DEVERR_TIMEOUT = range(4)
+MOE_DEVERR_NONE, MOE_DEVERR_EXPERT_ID, MOE_DEVERR_NOT_RESIDENT, MOE_DEVERR_TIMEOUT, MOE_DEVERR_RANGE = range(5)
 MOE_RENORM, MOE_LOGITS_GIVEN, MOE_IDS_GIVEN = 1, 2, 4
 MOE_PATH_AUTO, MOE_PATH_GEMV, MOE_PATH_TC = 0, 1, 2
 

@@ -90,6 +90,7 @@ int moe_read_device_error(void *ws, moe_stream_t stream, int32_t *code) {
     const char *what = v == MOE_DEVERR_EXPERT_ID     ? "expert id out of range"
                        : v == MOE_DEVERR_NOT_RESIDENT ? "active expert not resident in any slot"
                        : v == MOE_DEVERR_TIMEOUT      ? "bounded pipeline wait timed out"
+                       : v == MOE_DEVERR_RANGE        ? "activation outside FP16 range on the tensor-core path"
                                                       : "unknown device error";
     return moe::set_error(MOE_ERR_DEVICE, "device error %d: %s", v, what);
   }

@@ -1,14 +1,14 @@
 // A7 — router-weighted combine of the k expert outputs of each token, with
 // an optional residual: out[t] = bf16_rn(res[t] + sum_j w[t][j] * y[pos(t,j)]),
-// fp32 accumulation in increasing j (deterministic). One CTA per token; each
-// thread owns 8 consecutive hidden elements (16-byte loads and stores).
+// fp32 expert outputs, fp32 accumulation in increasing j (deterministic). One
+// CTA per token; each thread owns 8 consecutive hidden elements.
 #include "common.cuh"
 
 namespace moe {
 
 constexpr int CB_THREADS = 256;
 
-__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t *__restrict__ y,
+__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const float *__restrict__ y,
                                                               const float *__restrict__ topk_w,
                                                               const int32_t *__restrict__ pair_pos,
                                                               const uint16_t *residual, int k, int H,
@@ -35,11 +35,12 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t *__r
       const int pos = ps[j];
       if (pos < 0) continue;
       const float w = ws[j];
-      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + int64_t(pos) * H) + c);
-      acc[0] = fmaf(w, bf16_lo(v.x), acc[0]); acc[1] = fmaf(w, bf16_hi(v.x), acc[1]);
-      acc[2] = fmaf(w, bf16_lo(v.y), acc[2]); acc[3] = fmaf(w, bf16_hi(v.y), acc[3]);
-      acc[4] = fmaf(w, bf16_lo(v.z), acc[4]); acc[5] = fmaf(w, bf16_hi(v.z), acc[5]);
-      acc[6] = fmaf(w, bf16_lo(v.w), acc[6]); acc[7] = fmaf(w, bf16_hi(v.w), acc[7]);
+      const float4 *src = reinterpret_cast<const float4 *>(y + int64_t(pos) * H) + 2 * c;
+      const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
+      acc[0] = fmaf(w, v0.x, acc[0]); acc[1] = fmaf(w, v0.y, acc[1]);
+      acc[2] = fmaf(w, v0.z, acc[2]); acc[3] = fmaf(w, v0.w, acc[3]);
+      acc[4] = fmaf(w, v1.x, acc[4]); acc[5] = fmaf(w, v1.y, acc[5]);
+      acc[6] = fmaf(w, v1.z, acc[6]); acc[7] = fmaf(w, v1.w, acc[7]);
     }
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]); o.y = pack_bf16x2(acc[2], acc[3]);
@@ -50,7 +51,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t *__r
 
 }  // namespace moe
 
-extern "C" int moe_combine(const moe_bf16 *y, const float *topk_w, const int32_t *pair_pos,
+extern "C" int moe_combine(const float *y, const float *topk_w, const int32_t *pair_pos,
                            const moe_bf16 *residual, int T, int k, int H, moe_bf16 *out, moe_stream_t stream) {
   using namespace moe;
   if (T < 0 || k < 1 || k > MAX_K || H < 8 || H % 8)

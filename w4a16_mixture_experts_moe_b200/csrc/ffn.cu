@@ -13,14 +13,16 @@ constexpr int TC_MIN_ROWS_PER_EXPERT = 32;
 }  // namespace moe
 
 extern "C" size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path) {
-  (void)E; (void)H; (void)path;
+  (void)E; (void)path;
   if (T < 0 || k < 1 || I < 0) return moe::WS_HEADER;
-  return moe::WS_HEADER + moe::round256(size_t(T) * size_t(k) * size_t(I) * 2);
+  // header | h [T*k][I] 16-bit | x as FP16 [T][H] (tensor-core path)
+  return moe::WS_HEADER + moe::round256(size_t(T) * size_t(k) * size_t(I) * 2) +
+         moe::round256(size_t(T) * size_t(H) * 2);
 }
 
 extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair, const int32_t *offsets,
                                      const void *bank, int64_t record_bytes, const int32_t *expert_slot,
-                                     int n_slots, int T, int k, int E, int H, int I, int path, moe_bf16 *y,
+                                     int n_slots, int T, int k, int E, int H, int I, int path, float *y,
                                      void *ws, size_t ws_bytes, moe_stream_t stream) {
   using namespace moe;
   if (T < 0 || E < 1 || E > MAX_E || k < 1 || k > E || k > MAX_K)
@@ -58,6 +60,8 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
   a.off_gs = L.gate_s; a.off_us = L.up_s; a.off_ds = L.down_s;
   a.err = static_cast<int32_t *>(ws);
   a.h = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER);
+  a.x16 = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER +
+                                       round256(size_t(T) * size_t(k) * size_t(I) * 2));
   a.y = y;
   if (cudaMemsetAsync(a.err, 0, sizeof(int32_t), s) != cudaSuccess) return check_launch("moe_grouped_w4a16_ffn memset");
   if (T == 0) return MOE_OK;

@@ -16,8 +16,10 @@ struct FfnArgs {
   int n_slots;
   int T, k, E, H, I;
   int64_t off_gq, off_uq, off_dq, off_gs, off_us, off_ds;  // record layout
-  uint16_t *h;    // [P][I] workspace, sorted order
-  uint16_t *y;    // [P][H] output, sorted order
+  uint16_t *h;    // [P][I] workspace, sorted order (BF16 on the GEMV path; the
+                  // BF16-rounded value stored as FP16 on the tensor-core path)
+  uint16_t *x16;  // [T][H] FP16 copy of x (tensor-core path)
+  float *y;       // [P][H] fp32 expert outputs, sorted order
   int32_t *err;   // device error word
 };
 

@@ -130,9 +130,9 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
     for (int c = 0; c < 2; ++c) {
       const int r = n0 + 2 * t + c;
       if (r < cnt) {
-        uint16_t *yr = a.y + int64_t(lo + r) * a.H + row0 + g;
-        yr[0] = f_to_bf16(acc[c]);
-        yr[8] = f_to_bf16(acc[2 + c]);
+        float *yr = a.y + int64_t(lo + r) * a.H + row0 + g;
+        yr[0] = acc[c];
+        yr[8] = acc[2 + c];
       }
     }
   }

@@ -9,14 +9,25 @@
 //   warps 0-3  producers: gather the tile's token rows (cp.async, written in
 //              the 128-byte-swizzled K-major layout the MMA reads), copy the
 //              packed codes of their weight row, and dequantise them in
-//              registers to BF16 q*s (one rounding) straight into the
-//              swizzled A tile; fence.proxy.async, then arrive on `full`.
+//              registers to FP16 q*s straight into the swizzled A tile;
+//              fence.proxy.async, then arrive on `full`.
 //   warp 4     allocates tensor memory; one thread issues the MMAs
-//              (kind::f16, BF16 x BF16 -> fp32) and commits each stage back
-//              to its `empty` barrier and each finished tile to `tmem_full`.
+//              (kind::f16 with FP16 A and B, fp32 accumulate) and commits each
+//              stage back to its `empty` barrier and each finished tile to
+//              `tmem_full`.
 //   warps 5-8  epilogue: tcgen05.ld of the accumulator (lane = feature,
 //              column = token), SwiGLU (gate/up pass) or the plain output
 //              (down pass), BF16 stores to h / y in group-sorted row order.
+// Why FP16 operands: q*s has at most 3 + 8 significant bits (|q| <= 8 and an
+// 8-bit BF16 scale significand) and FP16 holds 11, so the dequantised weight
+// is exact; a BF16 activation (8 significant bits) converts to FP16 exactly
+// too. The MMA then sums exact products in fp32, the same arithmetic as the
+// GEMV path (scale applied to fp32 group sums). This holds while activations
+// stay within FP16's range (|v| <= 65504; values below 2^-17 round by at most
+// 2^-25) and scales are >= 2^-14; a pre-pass converts x to FP16 and flags
+// MOE_DEVERR_RANGE for an activation out of range. The gate/up epilogue
+// rounds h to BF16 (the method's A16 intermediate) and stores that value in
+// FP16, which again is exact.
 // Two accumulator buffers let the epilogue of tile i overlap the mainloop of
 // tile i+1. Every wait is bounded (about two seconds of %globaltimer); a wait
 // that runs out flags MOE_DEVERR_TIMEOUT and all roles drain and exit.
@@ -92,12 +103,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: fp32 accumulate, BF16 A and B, both K-major, M=128.
-__device__ __forceinline__ uint32_t idesc_bf16(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+// Instruction descriptor: fp32 accumulate (bits 4-5 = 1), FP16 A and B
+// (format fields 0), both K-major, N>>3 at bit 17, M>>4 at bit 24.
+__device__ __forceinline__ uint32_t idesc_f16(int n) {
+  return (1u << 4) | (uint32_t(n >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
@@ -266,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
       const uint16_t *src;
       if (GATEUP) {
         const int tok = valid ? a.sorted_pair[tl.lo + tl.n0 + i] / a.k : 0;
-        src = a.x + int64_t(tok) * KD + ks * BK;
+        src = a.x16 + int64_t(tok) * KD + ks * BK;
       } else {
         src = a.h + int64_t(valid ? tl.lo + tl.n0 + i : 0) * KD + ks * BK;
       }
@@ -282,7 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
       }
       cp_async_commit();
     }
-    const __nv_bfloat162 b136 = __floats2bfloat162_rn(136.0f, 136.0f);
+    const __half2 h1032 = __floats2half2_rn(1032.0f, 1032.0f);
     for (int it = 0; it < iters && ok; ++it) {
       const int nx = it + D;
       if (nx < iters) {
@@ -304,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
       for (int m = 0; m < C::NMAT; ++m) {
         const int64_t soff = (m == 0) ? (GATEUP ? a.off_gs : a.off_ds) : a.off_us;
         const uint16_t sbits = reinterpret_cast<const uint16_t *>(rec + soff)[int64_t(tl.f0 + i) * G + (ks * BK) / GROUP];
-        const __nv_bfloat162 sc = __bfloat162bfloat162(__ushort_as_bfloat16(sbits));
+        const __half2 sc = __half2half2(__float2half_rn(bf16_to_f(sbits)));
         const uint4 w0 = *reinterpret_cast<const uint4 *>(nib + (((2 * m) ^ rot) << 4));
         const uint4 w1 = *reinterpret_cast<const uint4 *>(nib + (((2 * m + 1) ^ rot) << 4));
         const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -314,9 +326,10 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
           uint32_t outp[4];
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
-            uint32_t tt = ((words[wd] >> (4 * p)) & 0x000F000Fu) | 0x43004300u;
-            __nv_bfloat162 q = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&tt), b136);
-            __nv_bfloat162 v = __hmul2(q, sc);
+            // OR-ing a nibble into FP16 1024.0 gives 1024 + u; minus 1032 = q
+            uint32_t tt = ((words[wd] >> (4 * p)) & 0x000F000Fu) | 0x64006400u;
+            __half2 q = __hsub2(*reinterpret_cast<__half2 *>(&tt), h1032);
+            __half2 v = __hmul2(q, sc);
             outp[p] = *reinterpret_cast<uint32_t *>(&v);
           }
           *reinterpret_cast<uint4 *>(arow + ((wd ^ (i & 7)) << 4)) = make_uint4(outp[0], outp[1], outp[2], outp[3]);
@@ -335,7 +348,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
         const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
         const Tile tl = decode_tile(sh, E, FT, t);
         const int n_mma = max(16, (tl.nvalid + 15) & ~15);
-        const uint32_t idesc = idesc_bf16(n_mma);
+        const uint32_t idesc = idesc_f16(n_mma);
         const int b = tl_i & 1;
         ok = wait_bounded(sh, &sh.tmem_empty[b], ((tl_i >> 1) & 1) ^ 1, a.err);
         if (!ok) break;
@@ -353,7 +366,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
             const uint64_t adesc = sw128_desc(smem_u32(st + m * C::A_BYTES));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              mma_bf16(d0 + m * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) != 0);
+              mma_f16(d0 + m * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) != 0);
           }
           mma_commit(&sh.empty[s]);
         }
@@ -388,7 +401,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
             const int j = j0 + jj;
             if (j < tl.nvalid) {
               const float gv = __uint_as_float(g[jj]), uv = __uint_as_float(u[jj]);
-              a.h[int64_t(tl.lo + tl.n0 + j) * NOUT + f] = f_to_bf16(silu_f(gv) * uv);
+              const float hv = bf16_to_f(f_to_bf16(silu_f(gv) * uv));  // A16: h is BF16
+              a.h[int64_t(tl.lo + tl.n0 + j) * NOUT + f] = __half_as_ushort(__float2half_rn(hv));
             }
           }
         } else {
@@ -396,7 +410,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int j = j0 + jj;
-            if (j < tl.nvalid) a.y[int64_t(tl.lo + tl.n0 + j) * NOUT + f] = f_to_bf16(__uint_as_float(g[jj]));
+            if (j < tl.nvalid) a.y[int64_t(tl.lo + tl.n0 + j) * NOUT + f] = __uint_as_float(g[jj]);
           }
         }
       }
@@ -414,6 +428,27 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
 }
 
 }  // namespace tc
+
+// x [T][H] BF16 -> FP16 copy for the tensor-core gate/up pass; flags values
+// outside FP16's finite range (they would become infinities).
+__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ x16,
+                                                       int64_t n8, int32_t *err) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + i);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+    bool bad = false;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float lo = bf16_lo(in[c]), hi = bf16_hi(in[c]);
+      bad |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+      const __half2 hv = __floats2half2_rn(lo, hi);
+      out[c] = *reinterpret_cast<const uint32_t *>(&hv);
+    }
+    if (bad) flag_error(err, MOE_DEVERR_RANGE);
+    reinterpret_cast<uint4 *>(x16)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
 
 static int sm_count() {
   static int cached[64] = {0};
@@ -439,6 +474,14 @@ int launch_ffn_tc(const FfnArgs &a, cudaStream_t s) {
   if (a.H % tc::BM || a.I % tc::BM)
     return set_error(MOE_ERR_UNSUPPORTED, "moe_grouped_w4a16_ffn: tensor-core path needs H, I multiples of 128");
   const int grid = sm_count();
+  {
+    const int64_t n8 = int64_t(a.T) * a.H / 8;
+    const int64_t want = (n8 + 255) / 256, cap = int64_t(grid) * 8;
+    const int blocks = int(want < cap ? (want > 0 ? want : 1) : cap);
+    x_to_f16_kernel<<<blocks, 256, 0, s>>>(a.x, a.x16, n8, a.err);
+    const int st0 = check_launch("moe_grouped_w4a16_ffn (tc x to fp16)");
+    if (st0 != MOE_OK) return st0;
+  }
   const size_t smem_gu = tc::Cfg<true>::SMEM, smem_dn = tc::Cfg<false>::SMEM;
   int st = allow_dynamic_smem(reinterpret_cast<const void *>(tc::tc_ffn_kernel<true>), smem_gu, "ffn tc gate/up");
   if (st != MOE_OK) return st;

@@ -67,12 +67,13 @@ __device__ int warp_exclusive_scan(const int32_t *in, int32_t *out, int E) {
 }
 
 // Stable rank of this thread's pair among the chunk's pairs of the same
-// expert; `wcnt` is [32 warps][E] shared scratch, `base` [E] the chunk's
-// first position per expert. Writes the outputs for valid pairs.
+// expert; `wcnt` is [warps][E] shared scratch, `base` [E] the chunk's first
+// position per expert. Writes the outputs for valid pairs.
 __device__ void chunk_scatter(int e, int p, int E, int32_t *wcnt, const int32_t *base, int32_t *sorted_pair,
                               int32_t *pair_pos, bool in_range) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+  const int nwarps = blockDim.x >> 5;
+  for (int i = threadIdx.x; i < nwarps * E; i += blockDim.x) wcnt[i] = 0;
   __syncthreads();
   const unsigned same = __match_any_sync(0xffffffffu, e);
   const int lane_rank = __popc(same & ((1u << lane) - 1u));
@@ -80,7 +81,7 @@ __device__ void chunk_scatter(int e, int p, int E, int32_t *wcnt, const int32_t 
   __syncthreads();
   for (int x = threadIdx.x; x < E; x += blockDim.x) {  // exclusive scan down each expert column
     int run = 0;
-    for (int w = 0; w < 32; ++w) {
+    for (int w = 0; w < nwarps; ++w) {
       const int c = wcnt[w * E + x];
       wcnt[w * E + x] = run;
       run += c;
@@ -96,7 +97,7 @@ __device__ void chunk_scatter(int e, int p, int E, int32_t *wcnt, const int32_t 
   }
 }
 
-// One-launch path: P <= GT_CHUNK.
+// One-launch path: P <= GT_CHUNK, one thread per pair (a single warp at T=1..4).
 __global__ void __launch_bounds__(GT_CHUNK) group_small_kernel(const int32_t *__restrict__ ids, int P, int E,
                                                                int32_t *counts, int32_t *offsets,
                                                                int32_t *sorted_pair, int32_t *pair_pos,
@@ -202,7 +203,8 @@ extern "C" int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E, in
   GroupWs g = group_ws(ws);
   if (cudaMemsetAsync(g.err, 0, sizeof(int32_t), s) != cudaSuccess) return check_launch("moe_group_tokens memset");
   if (P <= GT_CHUNK) {
-    group_small_kernel<<<1, GT_CHUNK, 0, s>>>(topk_ids, P, E, counts, offsets, sorted_pair, pair_pos, g.err);
+    const int threads = P <= 32 ? 32 : (P + 31) / 32 * 32;
+    group_small_kernel<<<1, threads, 0, s>>>(topk_ids, P, E, counts, offsets, sorted_pair, pair_pos, g.err);
     return check_launch("moe_group_tokens");
   }
   const int chunks = (P + GT_CHUNK - 1) / GT_CHUNK;

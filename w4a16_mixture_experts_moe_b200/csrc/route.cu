@@ -3,36 +3,58 @@
 // procedure is unchanged; Figure 1 caption: the original BF16 router selects
 // the experts).
 //
-// One CTA of 8 warps serves TT = 8 tokens: the tokens' activations are staged
-// in shared memory, each warp computes the logits of E/8 experts for all 8
-// tokens (fp32 sums, one BF16 rounding), then warp w runs softmax and a
-// shuffle-based top-k for token w. Lane l holds experts l, l+32, ...
-#include <float.h>
+// One thread-block cluster of 8 CTAs serves 8 tokens. CTA rank r computes the
+// logits of experts [r*EPC, (r+1)*EPC) (EPC = ceil(E/8)) for all 8 tokens:
+// the tokens' activations are staged in shared memory, each warp takes one
+// expert at a time with every lane's slice of the router row loaded at once
+// (fp32 sums, one BF16 rounding per logit). After a cluster barrier, CTA r
+// runs softmax and top-k for token r, reading the other CTAs' logits through
+// distributed shared memory; lane l holds experts l, l+32, ... and k rounds of
+// a shuffle argmax pick the experts. Splitting the router rows over 8 SMs
+// keeps a decode step (T of 1-64) from waiting on one SM's load latency.
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace moe {
 
-constexpr int RT_TOKENS = 8;
+constexpr int RT_TOKENS = 8;   // tokens per cluster (one per CTA for top-k)
+constexpr int RT_CLUSTER = 8;  // CTAs per cluster
 constexpr int RT_THREADS = 256;
+constexpr int RT_MAX_EPC = MAX_E / RT_CLUSTER;
 
 __device__ __forceinline__ bool key_better(float ka, int ea, float kb, int eb) {
   return ka > kb || (ka == kb && ea < eb);
 }
 
-__global__ void __launch_bounds__(RT_THREADS) route_topk_kernel(
-    const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, int T, int H, int E, int k,
-    const float *__restrict__ bias, int flags, uint16_t *__restrict__ logits,
-    int32_t *__restrict__ topk_ids, float *__restrict__ topk_w) {
+__device__ __forceinline__ float dot8(const uint4 &w, const uint4 &x, float a) {
+  a = fmaf(bf16_lo(w.x), bf16_lo(x.x), a); a = fmaf(bf16_hi(w.x), bf16_hi(x.x), a);
+  a = fmaf(bf16_lo(w.y), bf16_lo(x.y), a); a = fmaf(bf16_hi(w.y), bf16_hi(x.y), a);
+  a = fmaf(bf16_lo(w.z), bf16_lo(x.z), a); a = fmaf(bf16_hi(w.z), bf16_hi(x.z), a);
+  a = fmaf(bf16_lo(w.w), bf16_lo(x.w), a); a = fmaf(bf16_hi(w.w), bf16_hi(x.w), a);
+  return a;
+}
+
+__global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
+    route_topk_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, int T, int H, int E, int k,
+                      const float *__restrict__ bias, int flags, uint16_t *__restrict__ logits,
+                      int32_t *__restrict__ topk_ids, float *__restrict__ topk_w) {
   extern __shared__ __align__(16) unsigned char smem[];
-  float *keys = reinterpret_cast<float *>(smem);                          // [TT][E]
-  uint16_t *xs = reinterpret_cast<uint16_t *>(smem + RT_TOKENS * MAX_E * 4);  // [TT][H]
-  const int t0 = blockIdx.x * RT_TOKENS;
+  __shared__ float part[RT_TOKENS][RT_MAX_EPC];  // this CTA's logits (as fp32 of the BF16 value)
+  __shared__ float keys[MAX_E];                   // the token this CTA ranks
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = int(cluster.block_rank());
+  const int t0 = (blockIdx.x / RT_CLUSTER) * RT_TOKENS;
   const int nt = min(RT_TOKENS, T - t0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int EPC = (E + RT_CLUSTER - 1) / RT_CLUSTER;
+  const int e_lo = rank * EPC, e_hi = min(E, e_lo + EPC);
+  const bool given = flags & MOE_LOGITS_GIVEN;
 
-  if (!(flags & MOE_LOGITS_GIVEN)) {
-    // stage activations (16 B per thread-iteration)
+  if (!given) {
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [RT_TOKENS][H]
     const int chunks = H / 8;
     for (int c = threadIdx.x; c < RT_TOKENS * chunks; c += RT_THREADS) {
       const int tt = c / chunks, hc = c % chunks;
@@ -41,96 +63,105 @@ __global__ void __launch_bounds__(RT_THREADS) route_topk_kernel(
       reinterpret_cast<uint4 *>(xs + tt * H)[hc] = v;
     }
     __syncthreads();
-    for (int e = warp; e < E; e += RT_THREADS / 32) {
+    for (int e = e_lo + warp; e < e_hi; e += RT_THREADS / 32) {
       float acc[RT_TOKENS];
 #pragma unroll
       for (int tt = 0; tt < RT_TOKENS; ++tt) acc[tt] = 0.f;
       const uint4 *wrow = reinterpret_cast<const uint4 *>(wr + int64_t(e) * H);
-      for (int hc = lane; hc < chunks; hc += 32) {
+      int hc = lane;
+      for (; hc + 32 * 7 < chunks; hc += 32 * 8) {  // eight 16-byte loads in flight per lane
+        uint4 wv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) wv[u] = __ldg(wrow + hc + 32 * u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int tt = 0; tt < RT_TOKENS; ++tt)
+            acc[tt] = dot8(wv[u], reinterpret_cast<const uint4 *>(xs + tt * H)[hc + 32 * u], acc[tt]);
+      }
+      for (; hc < chunks; hc += 32) {
         const uint4 wv = __ldg(wrow + hc);
 #pragma unroll
-        for (int tt = 0; tt < RT_TOKENS; ++tt) {
-          const uint4 xv = reinterpret_cast<const uint4 *>(xs + tt * H)[hc];
-          float a = acc[tt];
-          a = fmaf(bf16_lo(wv.x), bf16_lo(xv.x), a); a = fmaf(bf16_hi(wv.x), bf16_hi(xv.x), a);
-          a = fmaf(bf16_lo(wv.y), bf16_lo(xv.y), a); a = fmaf(bf16_hi(wv.y), bf16_hi(xv.y), a);
-          a = fmaf(bf16_lo(wv.z), bf16_lo(xv.z), a); a = fmaf(bf16_hi(wv.z), bf16_hi(xv.z), a);
-          a = fmaf(bf16_lo(wv.w), bf16_lo(xv.w), a); a = fmaf(bf16_hi(wv.w), bf16_hi(xv.w), a);
-          acc[tt] = a;
-        }
+        for (int tt = 0; tt < RT_TOKENS; ++tt)
+          acc[tt] = dot8(wv, reinterpret_cast<const uint4 *>(xs + tt * H)[hc], acc[tt]);
       }
 #pragma unroll
       for (int tt = 0; tt < RT_TOKENS; ++tt) {
         float a = acc[tt];
 #pragma unroll
         for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == tt && tt < nt) {
+        if (lane == tt) {
           const uint16_t lb = f_to_bf16(a);
-          logits[int64_t(t0 + tt) * E + e] = lb;
-          keys[tt * E + e] = bf16_to_f(lb);
+          part[tt][e - e_lo] = bf16_to_f(lb);
+          if (tt < nt) logits[int64_t(t0 + tt) * E + e] = lb;
         }
       }
     }
-  } else {
-    for (int i = threadIdx.x; i < nt * E; i += RT_THREADS) keys[i] = bf16_to_f(logits[int64_t(t0) * E + i]);
   }
-  __syncthreads();
+  cluster.sync();  // every CTA's logits are in its shared memory
 
-  // ---- softmax + top-k, warp w handles token w
-  if (warp >= nt) return;
-  const int t = t0 + warp;
-  float *kr = keys + warp * E;
-  for (int e = lane; e < E; e += 32) {
-    float v = kr[e];
-    if (bias) v = v + bias[e];
-    if (v != v) v = -INFINITY;  // NaN never wins
-    kr[e] = v;
-  }
-  __syncwarp();
-  float mx = -INFINITY;
-  for (int e = lane; e < E; e += 32) mx = fmaxf(mx, kr[e]);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float sum = 0.f;
-  for (int e = lane; e < E; e += 32) sum += expf(kr[e] - mx);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-
-  int32_t *ids = topk_ids + int64_t(t) * k;
-  float *wout = topk_w + int64_t(t) * k;
-  float wsum = 0.f;
-  if (flags & MOE_IDS_GIVEN) {
-    for (int j = 0; j < k; ++j) {
-      const int e = ids[j];
-      const float p = (e >= 0 && e < E) ? expf(kr[e] - mx) / sum : 0.f;
-      wsum += p;
-      if (lane == 0) wout[j] = p;
-    }
-  } else {
-    uint32_t taken = 0;  // bit m: expert lane + 32m already chosen
-    for (int j = 0; j < k; ++j) {
-      float bk = -INFINITY;
-      int be = 0x7fffffff;
-      for (int m = 0; lane + 32 * m < E; ++m) {
-        const int e = lane + 32 * m;
-        if (!(taken >> m & 1u) && key_better(kr[e], e, bk, be)) { bk = kr[e]; be = e; }
+  // ---- softmax + top-k for token t0 + rank (warp 0 of each CTA)
+  const int t = t0 + rank;
+  if (warp == 0 && rank < nt) {
+    for (int e = lane; e < E; e += 32) {
+      float v;
+      if (given) {
+        v = bf16_to_f(logits[int64_t(t) * E + e]);
+      } else {
+        const float *remote = cluster.map_shared_rank(&part[0][0], e / EPC);
+        v = remote[rank * RT_MAX_EPC + (e % EPC)];
       }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (key_better(ok, oe, bk, be)) { bk = ok; be = oe; }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      const float p = expf(bk - mx) / sum;
-      wsum += p;
-      if (lane == 0) { ids[j] = be; wout[j] = p; }
+      if (bias) v = v + bias[e];
+      if (v != v) v = -INFINITY;  // NaN never wins
+      keys[e] = v;
     }
-  }
-  if (flags & MOE_RENORM) {
     __syncwarp();
-    for (int j = lane; j < k; j += 32) wout[j] = wout[j] / wsum;
+    float mx = -INFINITY;
+    for (int e = lane; e < E; e += 32) mx = fmaxf(mx, keys[e]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+    for (int e = lane; e < E; e += 32) sum += expf(keys[e] - mx);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+
+    int32_t *ids = topk_ids + int64_t(t) * k;
+    float *wout = topk_w + int64_t(t) * k;
+    float wsum = 0.f;
+    if (flags & MOE_IDS_GIVEN) {
+      for (int j = 0; j < k; ++j) {
+        const int e = ids[j];
+        const float p = (e >= 0 && e < E) ? expf(keys[e] - mx) / sum : 0.f;
+        wsum += p;
+        if (lane == 0) wout[j] = p;
+      }
+    } else {
+      uint32_t taken = 0;  // bit m: expert lane + 32m already chosen
+      for (int j = 0; j < k; ++j) {
+        float bk = -INFINITY;
+        int be = 0x7fffffff;
+        for (int m = 0; lane + 32 * m < E; ++m) {
+          const int e = lane + 32 * m;
+          if (!(taken >> m & 1u) && key_better(keys[e], e, bk, be)) { bk = keys[e]; be = e; }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+          const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+          if (key_better(ok, oe, bk, be)) { bk = ok; be = oe; }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        const float p = expf(bk - mx) / sum;
+        wsum += p;
+        if (lane == 0) { ids[j] = be; wout[j] = p; }
+      }
+    }
+    if (flags & MOE_RENORM) {
+      __syncwarp();
+      for (int j = lane; j < k; j += 32) wout[j] = wout[j] / wsum;
+    }
   }
+  cluster.sync();  // keep this CTA's shared memory alive until every reader is done
 }
 
 }  // namespace moe
@@ -151,14 +182,15 @@ extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T
     return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk: NULL pointer");
   if (need_x && (!aligned(x, 16) || !aligned(w_router, 16)))
     return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk: x and w_router must be 16-byte aligned");
-  const size_t smem = RT_TOKENS * MAX_E * 4 + (need_x ? size_t(RT_TOKENS) * H * 2 : 0);
-  if (smem > 227 * 1024) return set_error(MOE_ERR_SHAPE, "moe_route_topk: H=%d too large", H);
+  const size_t smem = need_x ? size_t(RT_TOKENS) * H * 2 : 0;
+  if (smem > 200 * 1024) return set_error(MOE_ERR_SHAPE, "moe_route_topk: H=%d too large", H);
   if (smem > 48 * 1024) {
     int st = allow_dynamic_smem(reinterpret_cast<const void *>(route_topk_kernel), smem, "moe_route_topk");
     if (st != MOE_OK) return st;
   }
-  const int blocks = (T + RT_TOKENS - 1) / RT_TOKENS;
-  route_topk_kernel<<<blocks, RT_THREADS, smem, as_stream(stream)>>>(x, w_router, T, H, E, k, bias, flags, logits,
-                                                                     topk_ids, topk_w);
+  const int64_t blocks = int64_t((T + RT_TOKENS - 1) / RT_TOKENS) * RT_CLUSTER;
+  if (blocks > 0x7fffffffLL) return set_error(MOE_ERR_SHAPE, "moe_route_topk: T too large");
+  route_topk_kernel<<<unsigned(blocks), RT_THREADS, smem, as_stream(stream)>>>(x, w_router, T, H, E, k, bias, flags,
+                                                                              logits, topk_ids, topk_w);
   return check_launch("moe_route_topk");
 }

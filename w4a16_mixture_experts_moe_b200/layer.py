@@ -67,7 +67,7 @@ class LayerBuffers:
         self.offsets = torch.empty(E + 1, dtype=torch.int32, **d)
         self.sorted_pair = torch.empty(max(P, 1), dtype=torch.int32, **d)
         self.pair_pos = torch.empty(max(P, 1), dtype=torch.int32, **d)
-        self.y = torch.empty(max(P, 1), H, dtype=torch.bfloat16, **d)
+        self.y = torch.empty(max(P, 1), H, dtype=torch.float32, **d)
         self.out = torch.empty(max(T, 1), H, dtype=torch.bfloat16, **d)
         self.group_ws_bytes = N.moe_group_workspace_size(T, k, E)
         self.group_ws = torch.zeros(self.group_ws_bytes, dtype=torch.uint8, **d)
