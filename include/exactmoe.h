@@ -161,6 +161,32 @@ int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E,
                      int32_t *sorted_pair, int32_t *pair_pos,
                      void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * moe_group_tokens without a workspace, for callers that cannot allocate
+ * device memory: code that runs under CUDA stream capture (where cudaMalloc
+ * is not allowed), or inside a host framework that owns every device
+ * allocation and offers no scratch space. (The paper has no counterpart;
+ * this exists only for such callers.)
+ *
+ * Same arguments, outputs and results as moe_group_tokens minus ws/ws_bytes.
+ * The scratch is a fixed array inside this library (about 64 KiB), which
+ * every GPU that loads the library holds until the process exits; it allows
+ * at most MOE_NOALLOC_MAX_PAIRS = T*k pairs (larger calls return
+ * MOE_ERR_SHAPE and launch nothing). This call allocates nothing and calls no
+ * cudaMalloc/cudaFree. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture. All calls share the one array: calls whose
+ * kernels overlap on the GPU (other streams, other host threads) race and
+ * corrupt each other's results, so serialise them. Device-side errors are not
+ * reported through a workspace word here: a pair with an out-of-range id gets
+ * pair_pos = -1, which the caller can check.
+ */
+#define MOE_NOALLOC_MAX_PAIRS 65536
+int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E,
+                             int32_t *counts, int32_t *offsets,
+                             int32_t *sorted_pair, int32_t *pair_pos,
+                             moe_stream_t stream);
+
 /* FFN execution paths. */
 #define MOE_PATH_AUTO 0 /* chosen from the average rows per expert, T*k/E */
 #define MOE_PATH_GEMV 1 /* decode-sized groups: weight-streaming, HBM-bound */

@@ -47,6 +47,7 @@ SIGNATURES = {
     "moe_route_topk": (_i, [_p, _p, _i, _i, _i, _i, _p, _i, _p, _p, _p, _p]),
     "moe_group_workspace_size": (_sz, [_i, _i, _i]),
     "moe_group_tokens": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
+    "moe_group_tokens_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
     "moe_ffn_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moe_grouped_w4a16_ffn": (_i, [_p, _p, _p, _p, _i64, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
@@ -133,6 +134,15 @@ def moe_group_workspace_size(T, k, E) -> int:
 def moe_group_tokens(topk_ids, T, k, E, counts, offsets, sorted_pair, pair_pos, ws, ws_bytes, stream=None):
     _check(lib.moe_group_tokens(_ptr(topk_ids), T, k, E, _ptr(counts), _ptr(offsets), _ptr(sorted_pair),
                                 _ptr(pair_pos), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def moe_group_tokens_noalloc(topk_ids, T, k, E, counts, offsets, sorted_pair, pair_pos, stream=None):
+    """moe_group_tokens with the library's fixed scratch (no workspace); see include/exactmoe.h."""
+    _check(lib.moe_group_tokens_noalloc(_ptr(topk_ids), T, k, E, _ptr(counts), _ptr(offsets), _ptr(sorted_pair),
+                                        _ptr(pair_pos), _stream(stream)))
+
+
+MOE_NOALLOC_MAX_PAIRS = 65536
 
 
 def moe_ffn_workspace_size(T, k, E, H, I, path=MOE_PATH_AUTO) -> int:

@@ -11,6 +11,8 @@
 //             counts scanned across warps) and writes sorted_pair/pair_pos.
 // With a single chunk (P <= 1024, every decode size) the three phases run in
 // one kernel launch.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -212,4 +214,56 @@ extern "C" int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E, in
   group_scan_kernel<<<1, MAX_E, 0, s>>>(chunks, E, g.table, counts, offsets);
   group_scatter_kernel<<<chunks, GT_CHUNK, 0, s>>>(topk_ids, P, E, g.table, sorted_pair, pair_pos);
   return check_launch("moe_group_tokens", 3);
+}
+
+// ---------------------------------------------------------------------------
+// Grouping for callers that cannot allocate device memory.
+//
+// Same computation and kernels as moe_group_tokens; the only difference is
+// where the scratch lives: a file-scope device array sized for at most
+// MOE_NOALLOC_MAX_PAIRS pairs and 256 experts, which every GPU that loads
+// this library keeps until the process exits. Host code must not use the
+// array's name as a device address (on the host it is only a stand-in), so
+// the address is looked up once per device with cudaGetSymbolAddress, with
+// that device current, on the first call made on it.
+namespace moe {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES =
+    WS_HEADER + size_t((MOE_NOALLOC_MAX_PAIRS + GT_CHUNK - 1) / GT_CHUNK) * MAX_E * sizeof(int32_t);
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+static int noalloc_scratch(void **out) {
+  static std::mutex mu;
+  static void *addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_group_tokens_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return set_error(MOE_ERR_UNSUPPORTED, "moe_group_tokens_noalloc: device %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return set_error(MOE_ERR_CUDA, "moe_group_tokens_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E, int32_t *counts,
+                                        int32_t *offsets, int32_t *sorted_pair, int32_t *pair_pos,
+                                        moe_stream_t stream) {
+  using namespace moe;
+  if (T < 0 || k < 1 || int64_t(T) * k > MOE_NOALLOC_MAX_PAIRS)
+    return set_error(MOE_ERR_SHAPE, "moe_group_tokens_noalloc: T*k = %lld pairs exceeds the fixed scratch limit of %d",
+                     (long long)(int64_t(T) * (k < 1 ? 1 : k)), MOE_NOALLOC_MAX_PAIRS);
+  void *ws = nullptr;
+  const int st = noalloc_scratch(&ws);
+  if (st != MOE_OK) return st;
+  return moe_group_tokens(topk_ids, T, k, E, counts, offsets, sorted_pair, pair_pos, ws, NOALLOC_SCRATCH_BYTES,
+                          stream);
 }
