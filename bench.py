@@ -47,8 +47,8 @@ def rec_bytes(h, i):
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--T", type=int, default=16)
     ap.add_argument("--layers", type=int, default=LAYERS)
@@ -132,9 +132,10 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        time.sleep(0.3)  # nvidia-smi needs a moment before its first sample
         return self
 
     def __exit__(self, *a):
@@ -202,29 +203,13 @@ class Stack:
         xs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
         return bufs, xs
 
-    def forward(self, bufs, xs, x_in, events=None):
-        """x_in -> layer 0 -> ... -> returns the output buffer. events: optional
-        list of (start, end) CUDA events recorded around each layer's FFN call."""
+    def forward(self, bufs, xs, x_in):
+        """x_in -> layer 0 -> ... -> returns the output buffer."""
         from w4a16_mixture_experts_moe_b200.layer import moe_layer_forward
-        M = self.M
-        H, I, E, K = self.H, self.I, self.E, self.K
         cur = x_in
         for l in range(self.layers):
             out = xs[l % 2] if cur is not xs[l % 2] else xs[(l + 1) % 2]
-            b = bufs[l]
-            T = b.T
-            if events is None:
-                moe_layer_forward(cur, self.routers[l], self.banks[l], b, flags=self.flags, residual=cur, out=out)
-            else:
-                M.moe_route_topk(cur, self.routers[l], T, H, E, K, None, self.flags, b.logits, b.topk_ids,
-                                 b.topk_w)
-                M.moe_group_tokens(b.topk_ids, T, K, E, b.counts, b.offsets, b.sorted_pair, b.pair_pos,
-                                   b.group_ws, b.group_ws_bytes)
-                events[l][0].record()
-                M.moe_grouped_w4a16_ffn(cur, b.sorted_pair, b.offsets, self.banks[l].ptr, self.banks[l].rec, None,
-                                        E, T, K, E, H, I, b.path, b.y, b.ffn_ws, b.ffn_ws_bytes)
-                events[l][1].record()
-                M.moe_combine(b.y, b.topk_w, b.pair_pos, cur, T, K, H, out)
+            moe_layer_forward(cur, self.routers[l], self.banks[l], bufs[l], flags=self.flags, residual=cur, out=out)
             cur = out
         return cur
 
@@ -283,16 +268,21 @@ def measure_T(stack, T, steps, warmup, world, want_e2e=True, want_roofline=True)
         ms_e2e = max_over_ranks(time_graph(torch, g2, steps, warmup), world)
         res["ms_e2e"] = ms_e2e
     if want_roofline:
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(stack.layers)]
-        per_call = []
-        reps = max(3, min(steps, 10))
-        for r in range(reps + 2):
-            stack.forward(bufs, xs, x_in, events=ev)
-            torch.cuda.synchronize()
-            if r >= 2:
-                per_call += [a.elapsed_time(b) for a, b in ev]
+        # The grouped FFN calls of all layers, replayed back to back from one
+        # graph on the buffers the step left behind (same routing, same
+        # launches as inside the step): CUDA events around the replays give
+        # the FFN call's device time.
+        g3 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g3, stream=stream):
+            for l in range(stack.layers):
+                b = bufs[l]
+                M.moe_grouped_w4a16_ffn(x_in if l == 0 else xs[(l - 1) % 2], b.sorted_pair, b.offsets,
+                                        stack.banks[l].ptr, stack.banks[l].rec, None, stack.E, T, stack.K, stack.E,
+                                        stack.H, stack.I, b.path, b.y, b.ffn_ws, b.ffn_ws_bytes)
+        ms_ffn_layers = time_graph(torch, g3, max(3, min(steps, 50)), 3)
+        del g3
         n_act = [int((b.counts > 0).sum().item()) for b in bufs]
-        res["ffn_ms_per_call"] = statistics.mean(per_call)
+        res["ffn_ms_per_call"] = ms_ffn_layers / stack.layers
         res["n_active_mean"] = statistics.mean(n_act)
         res["ffn_bytes_per_call"] = statistics.mean(n_act) * rec_bytes(stack.H, stack.I)
         res["ffn_flops_per_call"] = 6.0 * T * stack.K * stack.H * stack.I
@@ -451,10 +441,11 @@ def main_slotcache(a, rank, world, P):
     dst = torch.empty(probe_n * rec, dtype=torch.uint8, device="cuda")
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(2):
-        ev0.record(side)
-        for i in range(probe_n):
-            dst[i * rec:(i + 1) * rec].copy_(pool[i * rec:(i + 1) * rec], non_blocking=True)
-        ev1.record(side)
+        with torch.cuda.stream(side):
+            ev0.record(side)
+            for i in range(probe_n):
+                dst[i * rec:(i + 1) * rec].copy_(pool[i * rec:(i + 1) * rec], non_blocking=True)
+            ev1.record(side)
         side.synchronize()
     pinned_gbs = probe_n * rec / (ev0.elapsed_time(ev1) / 1e3) / 1e9
     del dst

@@ -21,8 +21,12 @@
  *  - Every call returns MOE_OK or an error status; moe_last_error() gives a
  *    message for the calling host thread. A failed argument check launches
  *    nothing. Errors found on the device (an expert id out of range, an expert
- *    that is not resident) are written to the first word of the workspace and
- *    read back with moe_read_device_error.
+ *    that is not resident) are written to the first word of the workspace,
+ *    where the first one stays until moe_read_device_error reads and clears
+ *    it; zero a workspace once before its first use.
+ *  - Kernels are launched with programmatic dependent launch, so each one's
+ *    launch overlaps the tail of the previous kernel on the stream; each
+ *    waits for its predecessor's results before reading them.
  *  - Shapes: hidden H and expert intermediate I are multiples of 128 (the
  *    quantisation group); 1 <= E <= 256 experts; 1 <= k <= min(E, 32).
  *
@@ -152,8 +156,8 @@ int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router,
  *   pair_pos    [T*k] int32 inverse: sorted_pair[pair_pos[p]] == p; -1 for a
  *               pair whose id is out of range (also flagged on the device).
  *   ws          workspace of at least moe_group_workspace_size(T, k, E) bytes,
- *               256-byte aligned. Word 0 is the device error word; this call
- *               clears it first.
+ *               256-byte aligned, zeroed once before first use. Word 0 is the
+ *               device error word.
  */
 size_t moe_group_workspace_size(int T, int k, int E);
 int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E,
@@ -211,12 +215,14 @@ int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E,
  *   y            [T*k][H] fp32, rows in sorted order (the expert outputs
  *                are kept unrounded until the combine).
  *   ws           at least moe_ffn_workspace_size(T, k, E, H, I, path) bytes,
- *                256-byte aligned; holds the error word and h.
- * Both paths form exact products x*(q*s) and sum them in fp32: the GEMV path
- * applies each group's scale to the fp32 partial sum of q*x over that group;
- * the tensor-core path dequantises q*s to FP16 (exact: at most 11 significant
- * bits) and feeds FP16 copies of the activations (exact for BF16 values up
- * to 65504 in magnitude; larger ones are flagged MOE_DEVERR_RANGE).
+ *                256-byte aligned, zeroed once before first use; holds the
+ *                error word, h and (tensor-core path) an FP16 copy of x.
+ * Both paths form exact products x*(q*s) and sum them in fp32, on FP16 copies
+ * of the activations (exact for BF16 values up to 65504 in magnitude; larger
+ * ones are flagged MOE_DEVERR_RANGE): the GEMV path multiplies FP16 codes q
+ * and applies each group's scale to the fp32 partial sum over that group; the
+ * tensor-core path dequantises q*s to FP16 (exact: at most 11 significant
+ * bits).
  */
 size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path);
 int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair,
@@ -225,6 +231,15 @@ int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair,
                           int n_slots, int T, int k, int E, int H, int I,
                           int path, float *y, void *ws, size_t ws_bytes,
                           moe_stream_t stream);
+
+/*
+ * Test hook for the failure path of the tensor-core FFN: the next `calls`
+ * tensor-core launches run with producers that never publish a stage, so the
+ * kernels' bounded waits (about two seconds each) run out, the kernels drain
+ * and return, and MOE_DEVERR_TIMEOUT is left in the workspace error word. The
+ * GPU context stays usable. Not for production use.
+ */
+int moe_debug_stall_next_tc_ffn(int calls);
 
 /*
  * A7 — router-weighted combine (implied by the MoE layer; the pages do not

@@ -142,7 +142,7 @@ def _group_gpu(M, ids, E):
     sp = torch.full((max(T * k, 1),), -7, dtype=torch.int32, device="cuda")
     pp = torch.full((max(T * k, 1),), -7, dtype=torch.int32, device="cuda")
     nb = M.moe_group_workspace_size(T, k, E)
-    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     M.moe_group_tokens(d, T, k, E, counts, offsets, sp, pp, ws, nb)
     code = M.moe_read_device_error(ws)
     return counts.cpu().numpy(), offsets.cpu().numpy(), sp.cpu().numpy()[:T * k], pp.cpu().numpy()[:T * k], code
@@ -194,7 +194,7 @@ def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None):
     offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
     sp = torch.empty(T * k, dtype=torch.int32, device="cuda")
     pp = torch.empty(T * k, dtype=torch.int32, device="cuda")
-    gws = torch.empty(M.moe_group_workspace_size(T, k, E), dtype=torch.uint8, device="cuda")
+    gws = torch.zeros(M.moe_group_workspace_size(T, k, E), dtype=torch.uint8, device="cuda")
     M.moe_group_tokens(d, T, k, E, counts, offsets, sp, pp, gws, gws.numel())
     y = torch.full((T * k, H), float("nan"), dtype=torch.float32, device="cuda")
     nb = M.moe_ffn_workspace_size(T, k, E, H, I, path)
@@ -203,8 +203,8 @@ def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None):
     M.moe_grouped_w4a16_ffn(x.cuda(), sp, offsets, bank.ptr, bank.rec, es, bank.n if n_slots is None else n_slots,
                             T, k, E, H, I, path, y, ws, nb)
     code = M.moe_read_device_error(ws)
-    # h is internal: BF16 on the GEMV path, the BF16-rounded value held in FP16 on the tensor-core path
-    h = ws[256:256 + T * k * I * 2].view(torch.float16 if path == M.MOE_PATH_TC else torch.bfloat16).view(T * k, I)
+    # h is internal: the BF16-rounded value held in FP16 (exact) on both paths
+    h = ws[256:256 + T * k * I * 2].view(torch.float16).view(T * k, I)
     return y.cpu().double().numpy(), h.float().cpu().double().numpy(), code
 
 
@@ -257,3 +257,29 @@ def test_combine(M, T, k, H, res):
     assert y.dtype == torch.float32
     assert_bf16_close(bf16_np(out), ref, "combine")
     assert np.mean(bf16_np(out) == ref) > 0.99   # one final rounding on both sides
+
+
+def test_tc_pipeline_wait_times_out_and_reports(M):
+    """Failure detection without a fault: the producers of one tensor-core FFN
+    call never publish a stage, every bounded wait runs out (~2 s), the kernels
+    drain and return, MOE_DEVERR_TIMEOUT is read back, and the next call on the
+    same context is correct again."""
+    import time
+    E, H, I, T, k = 4, 256, 256, 160, 2
+    gate = synth.normal_bf16((E, I, H), 0.02, 11)
+    up = synth.normal_bf16((E, I, H), 0.02, 12)
+    down = synth.normal_bf16((E, H, I), 0.02, 13)
+    bank = _make_bank(M, gate, up, down)
+    x = synth.activations(T, H, seed=14)
+    ids = np.stack([np.arange(k) + (t % (E - 1)) for t in range(T)]).astype(np.int32) % E
+    M.moe_debug_stall_next_tc_ffn(1)
+    t0 = time.time()
+    _, _, code = _ffn_gpu(M, bank, x, ids, k, M.MOE_PATH_TC, E)
+    assert code == M.MOE_DEVERR_TIMEOUT
+    assert time.time() - t0 < 30
+    y, _, code = _ffn_gpu(M, bank, x, ids, k, M.MOE_PATH_TC, E)
+    assert code == 0
+    experts = o.LazyQuantizedExperts(torch_weights_source(gate, up, down), E, H, I)
+    _, offsets, sp, _ = o.group_tokens(ids, E)
+    _, ref_y = o.grouped_ffn(x.double().numpy(), experts, sp, offsets, k)
+    assert_bf16_close(y, ref_y, "y after timeout")

@@ -50,6 +50,7 @@ SIGNATURES = {
     "moe_group_tokens_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
     "moe_ffn_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moe_grouped_w4a16_ffn": (_i, [_p, _p, _p, _p, _i64, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "moe_debug_stall_next_tc_ffn": (_i, [_i]),
     "moe_combine": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_read_device_error": (_i, [_p, _p, C.POINTER(C.c_int32)]),
     "slot_cache_create": (_i, [C.POINTER(_p), _i, _i, _i, _i64, _p, _p, _p]),
@@ -154,6 +155,11 @@ def moe_grouped_w4a16_ffn(x, sorted_pair, offsets, bank, record_bytes, expert_sl
     _check(lib.moe_grouped_w4a16_ffn(_ptr(x), _ptr(sorted_pair), _ptr(offsets), _ptr(bank), record_bytes,
                                      _ptr(expert_slot), n_slots, T, k, E, H, I, path, _ptr(y), _ptr(ws), ws_bytes,
                                      _stream(stream)))
+
+
+def moe_debug_stall_next_tc_ffn(calls: int):
+    """Test hook: the next `calls` tensor-core FFN launches time out on purpose."""
+    _check(lib.moe_debug_stall_next_tc_ffn(calls))
 
 
 def moe_combine(y, topk_w, pair_pos, residual, T, k, H, out, stream=None):

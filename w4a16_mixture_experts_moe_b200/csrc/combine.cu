@@ -15,6 +15,8 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const float *__rest
                                                               uint16_t *out) {
   __shared__ float ws[MAX_K];
   __shared__ int32_t ps[MAX_K];
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   if (threadIdx.x < k) {
     ws[threadIdx.x] = topk_w[int64_t(t) * k + threadIdx.x];
@@ -60,6 +62,8 @@ extern "C" int moe_combine(const float *y, const float *topk_w, const int32_t *p
   if (!y || !topk_w || !pair_pos || !out) return set_error(MOE_ERR_INVALID_ARG, "moe_combine: NULL pointer");
   if (!aligned(y, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)))
     return set_error(MOE_ERR_INVALID_ARG, "moe_combine: y, residual and out must be 16-byte aligned");
-  combine_kernel<<<T, CB_THREADS, 0, as_stream(stream)>>>(y, topk_w, pair_pos, residual, k, H, out);
+  cudaError_t e = launch_pdl(combine_kernel, dim3(T), dim3(CB_THREADS), 0, as_stream(stream), y, topk_w, pair_pos,
+                             residual, k, H, out);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_combine: %s", cudaGetErrorString(e));
   return check_launch("moe_combine");
 }

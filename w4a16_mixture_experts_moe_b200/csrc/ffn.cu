@@ -1,6 +1,8 @@
 // Entry point of the grouped W4A16 SwiGLU expert FFN (A5 + A6): argument
 // checks, workspace layout and the choice between the decode-sized GEMV path
 // and the prefill-sized tensor-core path.
+#include <atomic>
+
 #include "ffn.cuh"
 
 namespace moe {
@@ -10,7 +12,54 @@ static size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 // Average rows per expert at which the tensor-core path takes over.
 constexpr int TC_MIN_ROWS_PER_EXPERT = 32;
 
+// x [T][H] BF16 -> FP16 copy, the B operand of both gate/up paths (exact for
+// BF16 values of magnitude <= 65504); flags values outside FP16's finite range.
+__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ x16,
+                                                       int64_t n8, int32_t *err) {
+  pdl_trigger();
+  pdl_wait();
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + i);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+    bool bad = false;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float lo = bf16_lo(in[c]), hi = bf16_hi(in[c]);
+      bad |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+      const __half2 hv = __floats2half2_rn(lo, hi);
+      out[c] = *reinterpret_cast<const uint32_t *>(&hv);
+    }
+    if (bad) flag_error(err, MOE_DEVERR_RANGE);
+    reinterpret_cast<uint4 *>(x16)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+static std::atomic<int> g_tc_stall{0};
+
+int take_tc_stall() {
+  int v = g_tc_stall.load();
+  while (v > 0 && !g_tc_stall.compare_exchange_weak(v, v - 1)) {
+  }
+  return v > 0 ? 1 : 0;
+}
+
+int launch_x_to_f16(const FfnArgs &a, cudaStream_t s) {
+  const int64_t n8 = int64_t(a.T) * a.H / 8;
+  const int64_t want = (n8 + 255) / 256, cap = 148 * 8;
+  const int blocks = int(want < cap ? (want > 0 ? want : 1) : cap);
+  const cudaError_t e = launch_pdl(x_to_f16_kernel, dim3(blocks), dim3(256), 0, s, a.x, a.x16, n8, a.err);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (x to fp16): %s", cudaGetErrorString(e));
+  return check_launch("moe_grouped_w4a16_ffn (x to fp16)");
+}
+
 }  // namespace moe
+
+extern "C" int moe_debug_stall_next_tc_ffn(int calls) {
+  if (calls < 0) return moe::set_error(MOE_ERR_INVALID_ARG, "moe_debug_stall_next_tc_ffn: calls < 0");
+  moe::g_tc_stall.store(calls);
+  return MOE_OK;
+}
 
 extern "C" size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path) {
   (void)E; (void)path;
@@ -63,13 +112,14 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
   a.x16 = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER +
                                        round256(size_t(T) * size_t(k) * size_t(I) * 2));
   a.y = y;
-  if (cudaMemsetAsync(a.err, 0, sizeof(int32_t), s) != cudaSuccess) return check_launch("moe_grouped_w4a16_ffn memset");
+  a.stall = 0;
   if (T == 0) return MOE_OK;
 
   int chosen = path;
   if (path == MOE_PATH_AUTO)
     chosen = (int64_t(T) * k >= int64_t(TC_MIN_ROWS_PER_EXPERT) * E) ? MOE_PATH_TC : MOE_PATH_GEMV;
   if (chosen == MOE_PATH_TC) {
+    a.stall = take_tc_stall();
     st = launch_ffn_tc(a, s);
     if (st != MOE_ERR_UNSUPPORTED || path == MOE_PATH_TC) return st;
   }

@@ -16,12 +16,17 @@ struct FfnArgs {
   int n_slots;
   int T, k, E, H, I;
   int64_t off_gq, off_uq, off_dq, off_gs, off_us, off_ds;  // record layout
-  uint16_t *h;    // [P][I] workspace, sorted order (BF16 on the GEMV path; the
-                  // BF16-rounded value stored as FP16 on the tensor-core path)
-  uint16_t *x16;  // [T][H] FP16 copy of x (tensor-core path)
+  uint16_t *h;    // [P][I] workspace, sorted order: the BF16-rounded value
+                  // stored as FP16 (exact), the down pass's B operand
+  uint16_t *x16;  // [T][H] FP16 copy of x, the gate/up pass's B operand
   float *y;       // [P][H] fp32 expert outputs, sorted order
   int32_t *err;   // device error word
+  int stall;      // test hook: producers never publish a stage (bounded waits run out)
 };
+
+// Test hook state (moe_debug_stall_next_tc_ffn): number of tensor-core FFN
+// calls still to be launched with their producers stalled.
+int take_tc_stall();
 
 // Record of expert e, or nullptr (and the error flagged) if it has no slot.
 __device__ __forceinline__ const uint8_t *expert_record(const FfnArgs &a, int e) {
@@ -33,19 +38,6 @@ __device__ __forceinline__ const uint8_t *expert_record(const FfnArgs &a, int e)
   return a.bank + int64_t(slot) * a.rec;
 }
 
-// Offset-binary nibbles of one packed word -> four BF16x2 code pairs
-// (q_{2i}, q_{2i+1}), exact small integers: OR-ing a nibble into the
-// mantissa of BF16 128.0 gives 128 + u; subtracting 136 gives u - 8.
-__device__ __forceinline__ void dequant_codes(uint32_t w, uint32_t (&q)[4]) {
-  const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t t = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
-    __nv_bfloat162 v = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&t), bias);
-    q[i] = *reinterpret_cast<uint32_t *>(&v);
-  }
-}
-
 // Streaming 16-byte load that skips L1 (weights are read once).
 __device__ __forceinline__ uint4 ld_stream(const void *p) {
   uint4 v;
@@ -55,6 +47,7 @@ __device__ __forceinline__ uint4 ld_stream(const void *p) {
   return v;
 }
 
+int launch_x_to_f16(const FfnArgs &a, cudaStream_t s);
 int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s);
 int launch_ffn_tc(const FfnArgs &a, cudaStream_t s);
 

@@ -1,39 +1,79 @@
 // A5 + A6, decode-sized groups: a weight-streaming grouped GEMV on the
-// warp-level tensor-core MMA (mma.sync m16n8k16, BF16 in, fp32 out).
+// warp-level tensor-core MMA (mma.sync m16n8k16, FP16 in, fp32 out).
 //
 // A warp owns 16 output rows of one expert and walks K one 128-wide
-// quantisation group at a time. Lane (g, t) = (lane/4, lane%4) loads 16 bytes
-// (32 codes) of rows g and g+8 per matrix: the group's four lanes read 64
-// contiguous bytes of each row. The codes never leave registers: each packed
-// word turns into four BF16x2 code pairs (exact integers) that are used
+// quantisation group at a time (four groups per loop trip, so the load
+// offsets fold into the instructions). Lane (g, t) = (lane/4, lane%4) loads
+// 16 bytes (32 codes) of rows g and g+8 per matrix: the group's four lanes
+// read 64 contiguous bytes of each row. The codes never leave registers: each
+// packed word turns into four FP16x2 code pairs (exact integers) used
 // directly as A fragments. Because a dot product does not depend on the order
 // of its K terms, lane t's fragment slots are bound to ITS OWN 32 consecutive
 // k of the group (not the PTX fragment's k order); the B fragment (the
-// token's activations) is loaded with the same binding, so lane t reads 64
-// contiguous bytes of each token row. The fp32 sum of q*x over one group is
-// then multiplied by that row's group scale, so the dequantised weight q*s is
-// never rounded.
+// token's activations, FP16 copies) is loaded with the same binding, so lane t
+// reads 64 contiguous bytes of each token row. The fp32 sum of q*x over one
+// group is then multiplied by that row's group scale, so the dequantised
+// weight q*s is never rounded.
+//
+// Why FP16 operands: this kernel is bound by integer instructions spent
+// unpacking codes, and FP16's 10-bit mantissa lets a nibble sit at bits 4-7
+// of a half: one LOP3 yields (1024 + u) and another (1024 + 16u) for the next
+// code, with no shift. Codes and BF16 activations are exact in FP16 (the
+// activations while |x| <= 65504, which the FP16 copy of x checks).
+#include <cmath>
+
 #include "ffn.cuh"
 
 namespace moe {
 
 constexpr int GV_WARPS = 4;  // 64 rows per CTA
+constexpr int GV_UNROLL = 4;
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t x, uint32_t mask, uint32_t magic) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(mask), "r"(magic));  // (x & mask) | magic
+  return r;
+}
+
+// One packed word -> FP16x2 code pairs (q_{2i}, q_{2i+1}), i = 0..3. The word
+// holds k = 2i + h at bits 4(i + 4h): nibbles at bits 0-3/16-19 are pair 0,
+// 4-7/20-23 pair 1; after one right shift by 8, pairs 2 and 3 sit at the same
+// places. Low nibbles: (1024 + u) - 1032 = u - 8. High nibbles: (1024 + 16u)
+// / 16 - 72 = u - 8. Every step is exact in FP16.
+__device__ __forceinline__ void dequant_codes_f16(uint32_t w, uint32_t (&q)[4]) {
+  const __half2 lo_bias = __floats2half2_rn(1032.0f, 1032.0f);
+  const __half2 hi_scale = __floats2half2_rn(0.0625f, 0.0625f);
+  const __half2 hi_bias = __floats2half2_rn(-72.0f, -72.0f);
+  const uint32_t w8 = w >> 8;
+  uint32_t t0 = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+  uint32_t t1 = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
+  uint32_t t2 = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
+  uint32_t t3 = lop3_and_or(w8, 0x00F000F0u, 0x64006400u);
+  __half2 v0 = __hsub2(*reinterpret_cast<__half2 *>(&t0), lo_bias);
+  __half2 v1 = __hfma2(*reinterpret_cast<__half2 *>(&t1), hi_scale, hi_bias);
+  __half2 v2 = __hsub2(*reinterpret_cast<__half2 *>(&t2), lo_bias);
+  __half2 v3 = __hfma2(*reinterpret_cast<__half2 *>(&t3), hi_scale, hi_bias);
+  q[0] = *reinterpret_cast<uint32_t *>(&v0);
+  q[1] = *reinterpret_cast<uint32_t *>(&v1);
+  q[2] = *reinterpret_cast<uint32_t *>(&v2);
+  q[3] = *reinterpret_cast<uint32_t *>(&v3);
+}
+
 // One packed word of rows g (w0) and g+8 (w1) against the lane's 8 activations
-// (xb: BF16 pairs k 0-1, 2-3, 4-5, 6-7 of the word): two MMA k-steps.
+// (xb: FP16 pairs k 0-1, 2-3, 4-5, 6-7 of the word): two MMA k-steps.
 __device__ __forceinline__ void mma_word(float (&acc)[4], uint32_t w0, uint32_t w1, const uint4 &xb) {
   uint32_t q0[4], q1[4];
-  dequant_codes(w0, q0);
-  dequant_codes(w1, q1);
+  dequant_codes_f16(w0, q0);
+  dequant_codes_f16(w1, q1);
   mma_16816(acc, q0[0], q1[0], q0[1], q1[1], xb.x, xb.y);
   mma_16816(acc, q0[2], q1[2], q0[3], q1[3], xb.z, xb.w);
 }
@@ -45,28 +85,40 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint4 &w0, cons
   mma_word(acc, w0.w, w1.w, xb[3]);
 }
 
-// gate/up + SwiGLU: h[r][row] for the expert's rows r, 16 features per warp.
+// gate/up + SwiGLU: h[r][row] for the expert's rows r, 16 features per
+// slice. KS warps share a slice and split its groups (g % KS == the warp's
+// index within the slice) when there are few active experts; their partial
+// sums meet in shared memory. h is the BF16-rounded value stored as FP16
+// (exact), the down pass's B.
+template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArgs a) {
+  __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][8][32];
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.y;
   const int lo = a.offsets[e], cnt = a.offsets[e + 1] - lo;
   if (cnt <= 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int row0 = (blockIdx.x * GV_WARPS + warp) * 16;
-  if (row0 >= a.I) return;
+  const int sl = warp / KS, kq = warp % KS;  // row slice within the CTA, K part
+  const int row0 = (blockIdx.x * (GV_WARPS / KS) + sl) * 16;
+  if (blockIdx.x * (GV_WARPS / KS) * 16 >= a.I) return;  // whole CTA out of range (uniform)
+  const bool rows_ok = row0 < a.I;
   const uint8_t *rec = expert_record(a, e);
   if (!rec) return;
   const int H = a.H, KB = H / 2, G = H / GROUP;
-  const uint8_t *gq0 = rec + a.off_gq + int64_t(row0 + g) * KB + t * 16;
-  const uint8_t *uq0 = rec + a.off_uq + int64_t(row0 + g) * KB + t * 16;
-  const uint16_t *gs = reinterpret_cast<const uint16_t *>(rec + a.off_gs) + int64_t(row0 + g) * G;
-  const uint16_t *us = reinterpret_cast<const uint16_t *>(rec + a.off_us) + int64_t(row0 + g) * G;
+  const int rr = rows_ok ? row0 + g : 0;
+  const uint8_t *gq0 = rec + a.off_gq + int64_t(rr) * KB + t * 16;
+  const uint8_t *uq0 = rec + a.off_uq + int64_t(rr) * KB + t * 16;
+  const uint16_t *gs = reinterpret_cast<const uint16_t *>(rec + a.off_gs) + int64_t(rr) * G;
+  const uint16_t *us = reinterpret_cast<const uint16_t *>(rec + a.off_us) + int64_t(rr) * G;
 
   for (int n0 = 0; n0 < cnt; n0 += 8) {
     const bool ok = n0 + g < cnt;
     const int token = ok ? a.sorted_pair[lo + n0 + g] / a.k : 0;
-    const uint16_t *xr = a.x + int64_t(token) * H + t * 32;
+    const uint16_t *xr = a.x16 + int64_t(token) * H + t * 32;
     float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int grp = 0; grp < G; ++grp) {
+#pragma unroll GV_UNROLL
+    for (int grp = kq; grp < (rows_ok ? G : 0); grp += KS) {
       const uint4 g0 = ld_stream(gq0 + grp * 64), g1 = ld_stream(gq0 + 8 * KB + grp * 64);
       const uint4 u0 = ld_stream(uq0 + grp * 64), u1 = ld_stream(uq0 + 8 * KB + grp * 64);
       uint4 xb[4];
@@ -83,38 +135,61 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
       au[0] = fmaf(su0, pu[0], au[0]); au[1] = fmaf(su0, pu[1], au[1]);
       au[2] = fmaf(su1, pu[2], au[2]); au[3] = fmaf(su1, pu[3], au[3]);
     }
+    if (KS > 1) {  // K parts 1.. hand their sums to part 0 of the slice
+      __syncthreads();
+      if (kq > 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) { red[kq - 1][sl][c][lane] = ag[c]; red[kq - 1][sl][4 + c][lane] = au[c]; }
+      }
+      __syncthreads();
+      if (kq == 0) {
+#pragma unroll
+        for (int q = 0; q < KS - 1; ++q)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) { ag[c] += red[q][sl][c][lane]; au[c] += red[q][sl][4 + c][lane]; }
+      }
+    }
     // accumulator (c0, c1) = row g, tokens 2t, 2t+1; (c2, c3) = row g+8
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int r = n0 + 2 * t + c;
-      if (r < cnt) {
+      if (kq == 0 && rows_ok && r < cnt) {
         uint16_t *hr = a.h + int64_t(lo + r) * a.I + row0 + g;
-        hr[0] = f_to_bf16(silu_f(ag[c]) * au[c]);
-        hr[8] = f_to_bf16(silu_f(ag[2 + c]) * au[2 + c]);
+        hr[0] = __half_as_ushort(__float2half_rn(bf16_to_f(f_to_bf16(silu_f(ag[c]) * au[c]))));
+        hr[8] = __half_as_ushort(__float2half_rn(bf16_to_f(f_to_bf16(silu_f(ag[2 + c]) * au[2 + c]))));
       }
     }
   }
 }
 
-// down: y[r][row] = h[r] . Wd[row], 16 output features per warp.
+// down: y[r][row] = h[r] . Wd[row] (fp32), 16 output features per slice,
+// KS warps per slice as in the gate/up pass.
+template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs a) {
+  __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][4][32];
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.y;
   const int lo = a.offsets[e], cnt = a.offsets[e + 1] - lo;
   if (cnt <= 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int row0 = (blockIdx.x * GV_WARPS + warp) * 16;
-  if (row0 >= a.H) return;
+  const int sl = warp / KS, kq = warp % KS;
+  const int row0 = (blockIdx.x * (GV_WARPS / KS) + sl) * 16;
+  if (blockIdx.x * (GV_WARPS / KS) * 16 >= a.H) return;
+  const bool rows_ok = row0 < a.H;
   const uint8_t *rec = expert_record(a, e);
   if (!rec) return;
   const int I = a.I, KB = I / 2, G = I / GROUP;
-  const uint8_t *dq0 = rec + a.off_dq + int64_t(row0 + g) * KB + t * 16;
-  const uint16_t *ds = reinterpret_cast<const uint16_t *>(rec + a.off_ds) + int64_t(row0 + g) * G;
+  const int rr = rows_ok ? row0 + g : 0;
+  const uint8_t *dq0 = rec + a.off_dq + int64_t(rr) * KB + t * 16;
+  const uint16_t *ds = reinterpret_cast<const uint16_t *>(rec + a.off_ds) + int64_t(rr) * G;
 
   for (int n0 = 0; n0 < cnt; n0 += 8) {
     const bool ok = n0 + g < cnt;
     const uint16_t *hr = a.h + int64_t(lo + (ok ? n0 + g : 0)) * I + t * 32;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int grp = 0; grp < G; ++grp) {
+#pragma unroll GV_UNROLL
+    for (int grp = kq; grp < (rows_ok ? G : 0); grp += KS) {
       const uint4 w0 = ld_stream(dq0 + grp * 64), w1 = ld_stream(dq0 + 8 * KB + grp * 64);
       uint4 xb[4];
 #pragma unroll
@@ -126,10 +201,24 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
       acc[0] = fmaf(s0, p[0], acc[0]); acc[1] = fmaf(s0, p[1], acc[1]);
       acc[2] = fmaf(s1, p[2], acc[2]); acc[3] = fmaf(s1, p[3], acc[3]);
     }
+    if (KS > 1) {
+      __syncthreads();
+      if (kq > 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) red[kq - 1][sl][c][lane] = acc[c];
+      }
+      __syncthreads();
+      if (kq == 0) {
+#pragma unroll
+        for (int q = 0; q < KS - 1; ++q)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[c] += red[q][sl][c][lane];
+      }
+    }
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int r = n0 + 2 * t + c;
-      if (r < cnt) {
+      if (kq == 0 && rows_ok && r < cnt) {
         float *yr = a.y + int64_t(lo + r) * a.H + row0 + g;
         yr[0] = acc[c];
         yr[8] = acc[2 + c];
@@ -138,15 +227,38 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
   }
 }
 
-int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s) {
-  const int rows_per_cta = GV_WARPS * 16;
+template <int KS>
+static cudaError_t launch_gemv_pair(const FfnArgs &a, cudaStream_t s) {
+  const int rows_per_cta = (GV_WARPS / KS) * 16;
   dim3 g1((a.I + rows_per_cta - 1) / rows_per_cta, a.E);
-  gemv_gateup_kernel<<<g1, GV_WARPS * 32, 0, s>>>(a);
-  int st = check_launch("moe_grouped_w4a16_ffn (gemv gate/up)");
-  if (st != MOE_OK) return st;
+  cudaError_t e = launch_pdl(gemv_gateup_kernel<KS>, g1, dim3(GV_WARPS * 32), 0, s, a);
+  if (e != cudaSuccess) return e;
+  count_launches(1);
   dim3 g2((a.H + rows_per_cta - 1) / rows_per_cta, a.E);
-  gemv_down_kernel<<<g2, GV_WARPS * 32, 0, s>>>(a);
-  return check_launch("moe_grouped_w4a16_ffn (gemv down)");
+  e = launch_pdl(gemv_down_kernel<KS>, g2, dim3(GV_WARPS * 32), 0, s, a);
+  if (e == cudaSuccess) count_launches(1);
+  return e;
+}
+
+// Warps that share a 16-row slice, from the expected number of active experts
+// E (1 - (1 - k/E)^T): enough warps to keep every SM streaming when a decode
+// step touches few experts.
+static int pick_ksplit(const FfnArgs &a) {
+  const double miss = 1.0 - double(a.k) / double(a.E);
+  double n_act = double(a.E) * (1.0 - std::pow(miss, double(a.T)));
+  if (n_act < 1.0) n_act = 1.0;
+  const double warps = n_act * (a.I / 16);
+  const double want = 148.0 * 24.0;
+  return warps * 2 <= want ? 4 : (warps * 1.25 <= want ? 2 : 1);
+}
+
+int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s) {
+  int st = launch_x_to_f16(a, s);
+  if (st != MOE_OK) return st;
+  const int ks = pick_ksplit(a);
+  const cudaError_t e = ks == 4 ? launch_gemv_pair<4>(a, s) : ks == 2 ? launch_gemv_pair<2>(a, s) : launch_gemv_pair<1>(a, s);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (gemv): %s", cudaGetErrorString(e));
+  return check_launch("moe_grouped_w4a16_ffn (gemv)", 0);
 }
 
 }  // namespace moe

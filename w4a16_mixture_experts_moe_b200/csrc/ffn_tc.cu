@@ -2,9 +2,10 @@
 // tensor cores (tcgen05.mma, accumulators in tensor memory).
 //
 // "Swap AB": the MMA's M dimension is 128 output features of one expert, its
-// N dimension is up to 128 of that expert's tokens (rows of the group, so a
+// N dimension is up to 256 of that expert's tokens (rows of the group, so a
 // small group runs a narrow MMA instead of a padded one), and K walks the
-// input features 64 at a time. Per CTA (one per SM, persistent over a tile
+// input features 64 at a time. N = 256 halves the shared-memory traffic per
+// FLOP of the dequantised A tile, which bounds this kernel. Per CTA (one per SM, persistent over a tile
 // list built on the device from the group offsets):
 //   warps 0-3  producers: gather the tile's token rows (cp.async, written in
 //              the 128-byte-swizzled K-major layout the MMA reads), copy the
@@ -28,8 +29,9 @@
 // MOE_DEVERR_RANGE for an activation out of range. The gate/up epilogue
 // rounds h to BF16 (the method's A16 intermediate) and stores that value in
 // FP16, which again is exact.
-// Two accumulator buffers let the epilogue of tile i overlap the mainloop of
-// tile i+1. Every wait is bounded (about two seconds of %globaltimer); a wait
+// The down pass keeps two accumulator buffers so the epilogue of tile i
+// overlaps the mainloop of tile i+1; gate + up at N = 256 fill all 512
+// tensor-memory columns with one buffer. Every wait is bounded (about two seconds of %globaltimer); a wait
 // that runs out flags MOE_DEVERR_TIMEOUT and all roles drain and exit.
 #include "ffn.cuh"
 
@@ -37,24 +39,27 @@ namespace moe {
 namespace tc {
 
 constexpr int BM = 128;         // features per tile (MMA M)
-constexpr int BN = 128;         // max tokens per tile (MMA N)
+constexpr int BN = 256;         // max tokens per tile (MMA N)
 constexpr int BK = 64;          // K per stage (128 bytes of BF16 = one swizzle row)
-constexpr int STAGES = 3;
-constexpr int PRODUCERS = 128;  // warps 0-3
-constexpr int MMA_WARP = 4;
-constexpr int THREADS = 288;
+constexpr int MAX_STAGES = 5;
+constexpr int PRODUCERS = 256;  // warps 0-7: two threads per weight / token row of the tile
+constexpr int MMA_WARP = 8;
+constexpr int THREADS = 416;    // + warp 8 (MMA) + warps 9-12 (epilogue)
 constexpr uint64_t WAIT_NS = 2000000000ull;
 
 template <bool GATEUP>
 struct Cfg {
   static constexpr int NMAT = GATEUP ? 2 : 1;
   static constexpr int A_BYTES = BM * BK * 2;         // 16 KB per matrix
-  static constexpr int B_BYTES = BN * BK * 2;         // 16 KB
-  static constexpr int NIB_BYTES = PRODUCERS * 32 * NMAT;
+  static constexpr int B_BYTES = BN * BK * 2;         // 32 KB
+  static constexpr int NIB_BYTES = BM * 32 * NMAT;    // 32 bytes of codes per row and matrix
   static constexpr int STAGE_BYTES = NMAT * A_BYTES + B_BYTES + NIB_BYTES;
+  static constexpr int STAGES = GATEUP ? 3 : 4;       // as many as fit in 227 KB
   static constexpr int ACC_COLS = NMAT * BN;          // columns per accumulator buffer
-  static constexpr int TMEM_COLS = GATEUP ? 512 : 256;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int NBUF = TMEM_COLS / ACC_COLS;   // 1 (gate/up) or 2 (down) accumulator buffers
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 4096 /*tables, barriers*/;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -130,7 +135,7 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 
 // ------------------------------------------------------------------ shared state
 struct Shared {
-  uint64_t full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain;
+  uint64_t full[MAX_STAGES], empty[MAX_STAGES], tmem_full[2], tmem_empty[2], drain;
   uint32_t tmem_base;
   int32_t abort;
   int32_t total_tiles;
@@ -182,6 +187,7 @@ __device__ __forceinline__ Tile decode_tile(const Shared &sh, int E, int FT, int
 template <bool GATEUP>
 __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
   using C = Cfg<GATEUP>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Shared &sh = *reinterpret_cast<Shared *>(smem + STAGES * C::STAGE_BYTES);
@@ -192,11 +198,13 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
   const int FT = NOUT / BM;              // feature tiles per token tile
   const int KS = KD / BK;                // k-stages per tile
   const int G = KD / GROUP;
+  pdl_trigger();
+  pdl_wait();
 
   // ---- prologue: barriers, tensor memory, tile table
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&sh.full[s], PRODUCERS); mbar_init(&sh.empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&sh.tmem_full[b], 1); mbar_init(&sh.tmem_empty[b], 128); }
+    for (int b = 0; b < C::NBUF; ++b) { mbar_init(&sh.tmem_full[b], 1); mbar_init(&sh.tmem_empty[b], 128); }
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -247,46 +255,78 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
   const int iters = my_tiles * KS;
   auto stage_ptr = [&](int s) { return smem + s * C::STAGE_BYTES; };
 
-  if (warp < 4) {
+  if (warp < PRODUCERS / 32) {
     // ================================================================ producers
-    const int i = tid;  // weight row within the tile / token row within the tile
-    auto record = [&](int e) {
-      const int slot = a.expert_slot ? a.expert_slot[e] : e;
-      return a.bank + int64_t(slot) * a.rec;
-    };
-    auto issue = [&](int it) {
-      const int t = int(blockIdx.x) + (it / KS) * int(gridDim.x);
-      const int ks = it % KS;
+    // Thread (p, i): i = row of the tile (weight row f0+i and token row i),
+    // p = which half of the row's work: the matrix (gate/up pass) or the K
+    // half of the stage (down pass), and half of the token row's 8 chunks.
+    const int p = tid >> 7, i = tid & 127;
+    // per-tile state of the copy stream, refreshed when the stream enters a tile
+    int cur_tile = -1;
+    const uint8_t *qrow = nullptr;    // this thread's packed-code row
+    const uint16_t *srow = nullptr;   // its scale row
+    const uint16_t *brow_src[BN / BM] = {};
+    bool bvalid[BN / BM] = {};
+    auto enter_tile = [&](int tl_i) {
+      const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
       const Tile tl = decode_tile(sh, E, FT, t);
-      const uint8_t *rec = record(tl.e);
-      uint8_t *st = stage_ptr(it % STAGES);
-      // packed codes of row f0+i, this stage's 64 k = 32 bytes per matrix
-      const uint32_t nib = smem_u32(st + C::NMAT * C::A_BYTES + C::B_BYTES) + i * 32 * C::NMAT;
-      const int rot = (i >> 1) & (2 * C::NMAT - 1);
-      const int64_t rowoff = int64_t(tl.f0 + i) * (KD / 2) + ks * (BK / 2);
-      const uint8_t *q0 = rec + (GATEUP ? a.off_gq : a.off_dq) + rowoff;
-      cp_async16(nib + ((0 ^ rot) << 4), q0, 16);
-      cp_async16(nib + ((1 ^ rot) << 4), q0 + 16, 16);
-      if (GATEUP) {
-        const uint8_t *q1 = rec + a.off_uq + rowoff;
-        cp_async16(nib + ((2 ^ rot) << 4), q1, 16);
-        cp_async16(nib + ((3 ^ rot) << 4), q1 + 16, 16);
+      const int slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
+      const uint8_t *rec = a.bank + int64_t(slot) * a.rec;
+      const int m = GATEUP ? p : 0;
+      qrow = rec + (GATEUP ? (m ? a.off_uq : a.off_gq) : a.off_dq) + int64_t(tl.f0 + i) * (KD / 2);
+      srow = reinterpret_cast<const uint16_t *>(rec + (GATEUP ? (m ? a.off_us : a.off_gs) : a.off_ds)) +
+             int64_t(tl.f0 + i) * G;
+#pragma unroll
+      for (int h = 0; h < BN / BM; ++h) {
+        const int r = i + h * BM;
+        bvalid[h] = r < tl.nvalid;
+        if (GATEUP) {
+          const int tok = bvalid[h] ? a.sorted_pair[tl.lo + tl.n0 + r] / a.k : 0;
+          brow_src[h] = a.x16 + int64_t(tok) * KD;
+        } else {
+          brow_src[h] = a.h + int64_t(bvalid[h] ? tl.lo + tl.n0 + r : 0) * KD;
+        }
       }
-      // activation row i of the tile (token of the group, or h row), zero past the group
-      const uint32_t brow = smem_u32(st + C::NMAT * C::A_BYTES) + i * 128;
-      const bool valid = i < tl.nvalid;
-      const uint16_t *src;
-      if (GATEUP) {
-        const int tok = valid ? a.sorted_pair[tl.lo + tl.n0 + i] / a.k : 0;
-        src = a.x16 + int64_t(tok) * KD + ks * BK;
-      } else {
-        src = a.h + int64_t(valid ? tl.lo + tl.n0 + i : 0) * KD + ks * BK;
+      cur_tile = tl_i;
+    };
+    // per-tile state of the dequant stream (lags the copies by D stages)
+    int deq_tile = -1;
+    const uint16_t *deq_srow = nullptr;
+    auto scale_row = [&](int tl_i) {
+      const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + tl_i * int(gridDim.x));
+      const int slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
+      const uint8_t *rec = a.bank + int64_t(slot) * a.rec;
+      const int m = GATEUP ? p : 0;
+      return reinterpret_cast<const uint16_t *>(rec + (GATEUP ? (m ? a.off_us : a.off_gs) : a.off_ds)) +
+             int64_t(tl.f0 + i) * G;
+    };
+    // Copies of stage `it` (cp.async); its group scale is prefetched into L1
+    // so the dequant D stages later reads it without a long stall.
+    auto issue = [&](int it) {
+      if (it / KS != cur_tile) enter_tile(it / KS);
+      const int ks = it % KS;
+      uint8_t *st = stage_ptr(it % STAGES);
+      const uint32_t nib = smem_u32(st + C::NMAT * C::A_BYTES + C::B_BYTES);
+      if (GATEUP) {  // matrix p: 32 bytes (64 codes) of row i; chunk c at slot c ^ ((i >> 2) & 1)
+        const uint32_t d = nib + (p * BM + i) * 32;
+        const int r = (i >> 2) & 1;
+        cp_async16(d + ((0 ^ r) << 4), qrow + ks * (BK / 2), 16);
+        cp_async16(d + ((1 ^ r) << 4), qrow + ks * (BK / 2) + 16, 16);
+      } else {       // K half p: 16 bytes (32 codes) of row i
+        cp_async16(nib + (i * 2 + p) * 16, qrow + ks * (BK / 2) + p * 16, 16);
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) cp_async16(brow + ((c ^ (i & 7)) << 4), src + c * 8, valid ? 16 : 0);
+      for (int h = 0; h < BN / BM; ++h) {  // token rows i and i + 128
+        const uint32_t brow = smem_u32(st + C::NMAT * C::A_BYTES) + (i + h * BM) * 128;
+#pragma unroll
+        for (int c = 4 * p; c < 4 * p + 4; ++c)
+          cp_async16(brow + ((c ^ (i & 7)) << 4), brow_src[h] + ks * BK + c * 8, bvalid[h] ? 16 : 0);
+      }
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(srow + (ks * BK) / GROUP));
     };
-    constexpr int D = STAGES - 1;
+    constexpr int D = C::STAGES - 1;  // copy-ahead distance in stages
     bool ok = true;
+#pragma unroll
     for (int j = 0; j < D; ++j) {
       if (j < iters && ok) {
         ok = wait_bounded(sh, &sh.empty[j % STAGES], ((j / STAGES) & 1) ^ 1, a.err);
@@ -295,48 +335,67 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
       cp_async_commit();
     }
     const __half2 h1032 = __floats2half2_rn(1032.0f, 1032.0f);
+    const __half2 h16th = __floats2half2_rn(0.0625f, 0.0625f);
+    const __half2 hm72 = __floats2half2_rn(-72.0f, -72.0f);
+    // Per iteration: dequantise stage `it` and hand it to the MMA first, then
+    // refill the buffer the MMA has just finished with (stage it + D), so the
+    // dequant never waits for an MMA and the MMA finds each stage ready.
     for (int it = 0; it < iters && ok; ++it) {
+      if (it / KS != deq_tile) { deq_tile = it / KS; deq_srow = scale_row(deq_tile); }
+      const uint16_t sbits = deq_srow[((it % KS) * BK) / GROUP];  // L1 hit (prefetched)
+      cp_async_wait<D - 1>();  // the copies of stage `it` have landed
+      // dequantise this thread's codes of stage `it` into the swizzled A tile
+      uint8_t *st = stage_ptr(it % STAGES);
+      const uint8_t *nib = st + C::NMAT * C::A_BYTES + C::B_BYTES;
+      const __half2 sc = __half2half2(__float2half_rn(bf16_to_f(sbits)));
+      uint32_t words[8];
+      int nw, c0;
+      uint8_t *arow;
+      if (GATEUP) {
+        const uint8_t *src = nib + (p * BM + i) * 32;
+        const int r = (i >> 2) & 1;
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(src + ((0 ^ r) << 4));
+        const uint4 w1 = *reinterpret_cast<const uint4 *>(src + ((1 ^ r) << 4));
+        words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
+        words[4] = w1.x; words[5] = w1.y; words[6] = w1.z; words[7] = w1.w;
+        nw = 8; c0 = 0;
+        arow = st + p * C::A_BYTES + i * 128;
+      } else {
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(nib + (i * 2 + p) * 16);
+        words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
+        words[4] = words[5] = words[6] = words[7] = 0;
+        nw = 4; c0 = 4 * p;
+        arow = st + i * 128;
+      }
+#pragma unroll
+      for (int wd = 0; wd < 8; ++wd) {
+        if (wd >= nw) break;
+        // k = 2i + h sits at bits 4(i + 4h): OR-ing the nibbles at bits 0-3 /
+        // 16-19 into FP16 1024.0 gives (1024 + u), those at bits 4-7 / 20-23
+        // give (1024 + 16u); one shift by 8 brings pairs 2 and 3 to the same
+        // places. (1024 + u) - 1032 = q and (1024 + 16u) / 16 - 72 = q, exact.
+        const uint32_t w0 = words[wd], w8 = words[wd] >> 8;
+        const uint32_t tq[4] = {(w0 & 0x000F000Fu) | 0x64006400u, (w0 & 0x00F000F0u) | 0x64006400u,
+                                (w8 & 0x000F000Fu) | 0x64006400u, (w8 & 0x00F000F0u) | 0x64006400u};
+        uint32_t outp[4];
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+          const __half2 t2 = *reinterpret_cast<const __half2 *>(&tq[pp]);
+          const __half2 q = (pp & 1) ? __hfma2(t2, h16th, hm72) : __hsub2(t2, h1032);
+          __half2 v = __hmul2(q, sc);
+          outp[pp] = *reinterpret_cast<uint32_t *>(&v);
+        }
+        const int c = c0 + wd;
+        *reinterpret_cast<uint4 *>(arow + ((c ^ (i & 7)) << 4)) = make_uint4(outp[0], outp[1], outp[2], outp[3]);
+      }
+      fence_proxy_async();
+      if (!a.stall) mbar_arrive(&sh.full[it % STAGES]);
       const int nx = it + D;
       if (nx < iters) {
         ok = wait_bounded(sh, &sh.empty[nx % STAGES], ((nx / STAGES) & 1) ^ 1, a.err);
-        if (!ok) break;
-        issue(nx);
+        if (ok) issue(nx);
       }
       cp_async_commit();
-      cp_async_wait<D>();
-      // dequantise this thread's row(s) of stage `it` into the swizzled A tile(s)
-      const int t = int(blockIdx.x) + (it / KS) * int(gridDim.x);
-      const int ks = it % KS;
-      const Tile tl = decode_tile(sh, E, FT, t);
-      const uint8_t *rec = record(tl.e);
-      uint8_t *st = stage_ptr(it % STAGES);
-      const uint8_t *nib = st + C::NMAT * C::A_BYTES + C::B_BYTES + i * 32 * C::NMAT;
-      const int rot = (i >> 1) & (2 * C::NMAT - 1);
-#pragma unroll
-      for (int m = 0; m < C::NMAT; ++m) {
-        const int64_t soff = (m == 0) ? (GATEUP ? a.off_gs : a.off_ds) : a.off_us;
-        const uint16_t sbits = reinterpret_cast<const uint16_t *>(rec + soff)[int64_t(tl.f0 + i) * G + (ks * BK) / GROUP];
-        const __half2 sc = __half2half2(__float2half_rn(bf16_to_f(sbits)));
-        const uint4 w0 = *reinterpret_cast<const uint4 *>(nib + (((2 * m) ^ rot) << 4));
-        const uint4 w1 = *reinterpret_cast<const uint4 *>(nib + (((2 * m + 1) ^ rot) << 4));
-        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        uint8_t *arow = st + m * C::A_BYTES + i * 128;
-#pragma unroll
-        for (int wd = 0; wd < 8; ++wd) {
-          uint32_t outp[4];
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            // OR-ing a nibble into FP16 1024.0 gives 1024 + u; minus 1032 = q
-            uint32_t tt = ((words[wd] >> (4 * p)) & 0x000F000Fu) | 0x64006400u;
-            __half2 q = __hsub2(*reinterpret_cast<__half2 *>(&tt), h1032);
-            __half2 v = __hmul2(q, sc);
-            outp[p] = *reinterpret_cast<uint32_t *>(&v);
-          }
-          *reinterpret_cast<uint4 *>(arow + ((wd ^ (i & 7)) << 4)) = make_uint4(outp[0], outp[1], outp[2], outp[3]);
-        }
-      }
-      fence_proxy_async();
-      mbar_arrive(&sh.full[it % STAGES]);
     }
     cp_async_wait<0>();
   } else if (warp == MMA_WARP) {
@@ -349,8 +408,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
         const Tile tl = decode_tile(sh, E, FT, t);
         const int n_mma = max(16, (tl.nvalid + 15) & ~15);
         const uint32_t idesc = idesc_f16(n_mma);
-        const int b = tl_i & 1;
-        ok = wait_bounded(sh, &sh.tmem_empty[b], ((tl_i >> 1) & 1) ^ 1, a.err);
+        const int b = tl_i % C::NBUF;
+        ok = wait_bounded(sh, &sh.tmem_empty[b], ((tl_i / C::NBUF) & 1) ^ 1, a.err);
         if (!ok) break;
         tc_fence_after();
         const uint32_t d0 = tmem + b * C::ACC_COLS;
@@ -384,8 +443,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
     for (int tl_i = 0; tl_i < my_tiles; ++tl_i) {
       const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
       const Tile tl = decode_tile(sh, E, FT, t);
-      const int b = tl_i & 1;
-      if (!wait_bounded(sh, &sh.tmem_full[b], (tl_i >> 1) & 1, a.err)) break;
+      const int b = tl_i % C::NBUF;
+      if (!wait_bounded(sh, &sh.tmem_full[b], (tl_i / C::NBUF) & 1, a.err)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + (uint32_t(q * 32) << 16) + b * C::ACC_COLS;
       const int f = tl.f0 + frow;
@@ -429,27 +488,6 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
 
 }  // namespace tc
 
-// x [T][H] BF16 -> FP16 copy for the tensor-core gate/up pass; flags values
-// outside FP16's finite range (they would become infinities).
-__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ x16,
-                                                       int64_t n8, int32_t *err) {
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + i);
-    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out[4];
-    bool bad = false;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float lo = bf16_lo(in[c]), hi = bf16_hi(in[c]);
-      bad |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
-      const __half2 hv = __floats2half2_rn(lo, hi);
-      out[c] = *reinterpret_cast<const uint32_t *>(&hv);
-    }
-    if (bad) flag_error(err, MOE_DEVERR_RANGE);
-    reinterpret_cast<uint4 *>(x16)[i] = make_uint4(out[0], out[1], out[2], out[3]);
-  }
-}
-
 static int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -474,23 +512,19 @@ int launch_ffn_tc(const FfnArgs &a, cudaStream_t s) {
   if (a.H % tc::BM || a.I % tc::BM)
     return set_error(MOE_ERR_UNSUPPORTED, "moe_grouped_w4a16_ffn: tensor-core path needs H, I multiples of 128");
   const int grid = sm_count();
-  {
-    const int64_t n8 = int64_t(a.T) * a.H / 8;
-    const int64_t want = (n8 + 255) / 256, cap = int64_t(grid) * 8;
-    const int blocks = int(want < cap ? (want > 0 ? want : 1) : cap);
-    x_to_f16_kernel<<<blocks, 256, 0, s>>>(a.x, a.x16, n8, a.err);
-    const int st0 = check_launch("moe_grouped_w4a16_ffn (tc x to fp16)");
-    if (st0 != MOE_OK) return st0;
-  }
+  int st0 = launch_x_to_f16(a, s);
+  if (st0 != MOE_OK) return st0;
   const size_t smem_gu = tc::Cfg<true>::SMEM, smem_dn = tc::Cfg<false>::SMEM;
   int st = allow_dynamic_smem(reinterpret_cast<const void *>(tc::tc_ffn_kernel<true>), smem_gu, "ffn tc gate/up");
   if (st != MOE_OK) return st;
   st = allow_dynamic_smem(reinterpret_cast<const void *>(tc::tc_ffn_kernel<false>), smem_dn, "ffn tc down");
   if (st != MOE_OK) return st;
-  tc::tc_ffn_kernel<true><<<grid, tc::THREADS, smem_gu, s>>>(a);
+  cudaError_t e = launch_pdl(tc::tc_ffn_kernel<true>, dim3(grid), dim3(tc::THREADS), smem_gu, s, a);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (tc gate/up): %s", cudaGetErrorString(e));
   st = check_launch("moe_grouped_w4a16_ffn (tc gate/up)");
   if (st != MOE_OK) return st;
-  tc::tc_ffn_kernel<false><<<grid, tc::THREADS, smem_dn, s>>>(a);
+  e = launch_pdl(tc::tc_ffn_kernel<false>, dim3(grid), dim3(tc::THREADS), smem_dn, s, a);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (tc down): %s", cudaGetErrorString(e));
   return check_launch("moe_grouped_w4a16_ffn (tc down)");
 }
 

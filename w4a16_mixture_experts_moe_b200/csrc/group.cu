@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(GT_CHUNK) group_small_kernel(const int32_t *__
                                                                int32_t *counts, int32_t *offsets,
                                                                int32_t *sorted_pair, int32_t *pair_pos,
                                                                int32_t *err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t hist[MAX_E + 1];
   __shared__ int32_t base[MAX_E];
   __shared__ int32_t wcnt[32 * MAX_E];
@@ -128,6 +130,8 @@ __global__ void __launch_bounds__(GT_CHUNK) group_small_kernel(const int32_t *__
 
 __global__ void __launch_bounds__(GT_CHUNK) group_hist_kernel(const int32_t *__restrict__ ids, int P, int E,
                                                               int32_t *table, int32_t *err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t hist[MAX_E];
   for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
@@ -140,6 +144,8 @@ __global__ void __launch_bounds__(GT_CHUNK) group_hist_kernel(const int32_t *__r
 
 __global__ void __launch_bounds__(MAX_E) group_scan_kernel(int chunks, int E, int32_t *table, int32_t *counts,
                                                           int32_t *offsets) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t tot[MAX_E];
   __shared__ int32_t off[MAX_E];
   const int x = threadIdx.x;
@@ -168,6 +174,8 @@ __global__ void __launch_bounds__(MAX_E) group_scan_kernel(int chunks, int E, in
 __global__ void __launch_bounds__(GT_CHUNK) group_scatter_kernel(const int32_t *__restrict__ ids, int P, int E,
                                                                  const int32_t *table, int32_t *sorted_pair,
                                                                  int32_t *pair_pos) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t base[MAX_E];
   __shared__ int32_t wcnt[32 * MAX_E];
   for (int i = threadIdx.x; i < E; i += blockDim.x) base[i] = table[blockIdx.x * E + i];
@@ -203,16 +211,21 @@ extern "C" int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E, in
   cudaStream_t s = as_stream(stream);
   const int P = int(P64);
   GroupWs g = group_ws(ws);
-  if (cudaMemsetAsync(g.err, 0, sizeof(int32_t), s) != cudaSuccess) return check_launch("moe_group_tokens memset");
+  cudaError_t e;
   if (P <= GT_CHUNK) {
     const int threads = P <= 32 ? 32 : (P + 31) / 32 * 32;
-    group_small_kernel<<<1, threads, 0, s>>>(topk_ids, P, E, counts, offsets, sorted_pair, pair_pos, g.err);
+    e = launch_pdl(group_small_kernel, dim3(1), dim3(threads), 0, s, topk_ids, P, E, counts, offsets, sorted_pair,
+                   pair_pos, g.err);
+    if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_group_tokens: %s", cudaGetErrorString(e));
     return check_launch("moe_group_tokens");
   }
   const int chunks = (P + GT_CHUNK - 1) / GT_CHUNK;
-  group_hist_kernel<<<chunks, GT_CHUNK, 0, s>>>(topk_ids, P, E, g.table, g.err);
-  group_scan_kernel<<<1, MAX_E, 0, s>>>(chunks, E, g.table, counts, offsets);
-  group_scatter_kernel<<<chunks, GT_CHUNK, 0, s>>>(topk_ids, P, E, g.table, sorted_pair, pair_pos);
+  e = launch_pdl(group_hist_kernel, dim3(chunks), dim3(GT_CHUNK), 0, s, topk_ids, P, E, g.table, g.err);
+  if (e == cudaSuccess) e = launch_pdl(group_scan_kernel, dim3(1), dim3(MAX_E), 0, s, chunks, E, g.table, counts, offsets);
+  if (e == cudaSuccess)
+    e = launch_pdl(group_scatter_kernel, dim3(chunks), dim3(GT_CHUNK), 0, s, topk_ids, P, E,
+                   static_cast<const int32_t *>(g.table), sorted_pair, pair_pos);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_group_tokens: %s", cudaGetErrorString(e));
   return check_launch("moe_group_tokens", 3);
 }
 

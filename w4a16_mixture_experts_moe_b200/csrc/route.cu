@@ -45,6 +45,8 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
   __shared__ float part[RT_TOKENS][RT_MAX_EPC];  // this CTA's logits (as fp32 of the BF16 value)
   __shared__ float keys[MAX_E];                   // the token this CTA ranks
   cg::cluster_group cluster = cg::this_cluster();
+  pdl_trigger();
+  pdl_wait();
   const int rank = int(cluster.block_rank());
   const int t0 = (blockIdx.x / RT_CLUSTER) * RT_TOKENS;
   const int nt = min(RT_TOKENS, T - t0);
@@ -56,6 +58,17 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
   if (!given) {
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [RT_TOKENS][H]
     const int chunks = H / 8;
+    // this warp's first router row: its loads go out before the activations'
+    // so the two round trips overlap
+    constexpr int PRE = 8;
+    uint4 wpre[PRE];
+    const int e_first = e_lo + warp;
+#pragma unroll
+    for (int u = 0; u < PRE; ++u) {
+      const int hc = lane + 32 * u;
+      wpre[u] = (e_first < e_hi && hc < chunks) ? __ldg(reinterpret_cast<const uint4 *>(wr + int64_t(e_first) * H) + hc)
+                                                 : make_uint4(0, 0, 0, 0);
+    }
     for (int c = threadIdx.x; c < RT_TOKENS * chunks; c += RT_THREADS) {
       const int tt = c / chunks, hc = c % chunks;
       uint4 v = make_uint4(0, 0, 0, 0);
@@ -71,8 +84,9 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
       int hc = lane;
       for (; hc + 32 * 7 < chunks; hc += 32 * 8) {  // eight 16-byte loads in flight per lane
         uint4 wv[8];
+        const bool prefetched = (e == e_first && hc == lane);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) wv[u] = __ldg(wrow + hc + 32 * u);
+        for (int u = 0; u < 8; ++u) wv[u] = prefetched ? wpre[u] : __ldg(wrow + hc + 32 * u);
 #pragma unroll
         for (int u = 0; u < 8; ++u)
 #pragma unroll
@@ -190,7 +204,8 @@ extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T
   }
   const int64_t blocks = int64_t((T + RT_TOKENS - 1) / RT_TOKENS) * RT_CLUSTER;
   if (blocks > 0x7fffffffLL) return set_error(MOE_ERR_SHAPE, "moe_route_topk: T too large");
-  route_topk_kernel<<<unsigned(blocks), RT_THREADS, smem, as_stream(stream)>>>(x, w_router, T, H, E, k, bias, flags,
-                                                                              logits, topk_ids, topk_w);
+  const cudaError_t e = launch_pdl(route_topk_kernel, dim3(unsigned(blocks)), dim3(RT_THREADS), smem,
+                                   as_stream(stream), x, w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_route_topk: %s", cudaGetErrorString(e));
   return check_launch("moe_route_topk");
 }
