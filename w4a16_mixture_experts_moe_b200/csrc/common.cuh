@@ -52,7 +52,10 @@ __device__ __forceinline__ void flag_error(int32_t *err, int32_t code) {
   if (err) atomicCAS(err, 0, code);
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// SiLU with CUDA's fast exponential and fast divide (a few ulp in fp32, far
+// below the BF16 rounding of h that follows; for g < -88 the denominator is
+// +inf and the result 0).
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // Programmatic dependent launch: every hot-path kernel lets the next kernel of
 // the stream be scheduled as soon as all of its own CTAs are running

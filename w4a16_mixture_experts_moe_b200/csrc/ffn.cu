@@ -12,27 +12,51 @@ static size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 // Average rows per expert at which the tensor-core path takes over.
 constexpr int TC_MIN_ROWS_PER_EXPERT = 32;
 
-// x [T][H] BF16 -> FP16 copy, the B operand of both gate/up paths (exact for
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, bool &bad) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float lo = bf16_lo(in[c]), hi = bf16_hi(in[c]);
+    bad |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+    const __half2 hv = __floats2half2_rn(lo, hi);
+    out[c] = *reinterpret_cast<const uint32_t *>(&hv);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// x [T][H] BF16 -> FP16 copy, the decode path's gate/up input (exact for
 // BF16 values of magnitude <= 65504); flags values outside FP16's finite range.
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ x16,
                                                        int64_t n8, int32_t *err) {
   pdl_trigger();
   pdl_wait();
+  bool bad = false;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x)
+    reinterpret_cast<uint4 *>(x16)[i] = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4 *>(x) + i), bad);
+  if (bad) flag_error(err, MOE_DEVERR_RANGE);
+}
+
+// xs[r] = FP16(x[sorted_pair[r] / k]) for the P rows in group order: the
+// tensor-core gate/up pass then loads each token tile of an expert as one
+// contiguous block of rows.
+__global__ void __launch_bounds__(256) gather_x_f16_kernel(const uint16_t *__restrict__ x,
+                                                           const int32_t *__restrict__ sorted_pair, int k, int T,
+                                                           int H8, int64_t n8, uint16_t *__restrict__ xs,
+                                                           int32_t *err) {
+  pdl_trigger();
+  pdl_wait();
+  bool bad = false;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + i);
-    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out[4];
-    bool bad = false;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float lo = bf16_lo(in[c]), hi = bf16_hi(in[c]);
-      bad |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
-      const __half2 hv = __floats2half2_rn(lo, hi);
-      out[c] = *reinterpret_cast<const uint32_t *>(&hv);
-    }
-    if (bad) flag_error(err, MOE_DEVERR_RANGE);
-    reinterpret_cast<uint4 *>(x16)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    const int64_t r = i / H8;
+    const int c = int(i - r * H8);
+    const int t = sorted_pair[r] / k;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (t >= 0 && t < T) v = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4 *>(x + int64_t(t) * H8 * 8) + c), bad);
+    else flag_error(err, MOE_DEVERR_EXPERT_ID);
+    reinterpret_cast<uint4 *>(xs)[i] = v;
   }
+  if (bad) flag_error(err, MOE_DEVERR_RANGE);
 }
 
 static std::atomic<int> g_tc_stall{0};
@@ -53,6 +77,16 @@ int launch_x_to_f16(const FfnArgs &a, cudaStream_t s) {
   return check_launch("moe_grouped_w4a16_ffn (x to fp16)");
 }
 
+int launch_gather_x_f16(const FfnArgs &a, cudaStream_t s) {
+  const int64_t n8 = int64_t(a.T) * a.k * a.H / 8;
+  const int64_t want = (n8 + 255) / 256, cap = 148 * 8;
+  const int blocks = int(want < cap ? (want > 0 ? want : 1) : cap);
+  const cudaError_t e =
+      launch_pdl(gather_x_f16_kernel, dim3(blocks), dim3(256), 0, s, a.x, a.sorted_pair, a.k, a.T, a.H / 8, n8, a.xs, a.err);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (gather x): %s", cudaGetErrorString(e));
+  return check_launch("moe_grouped_w4a16_ffn (gather x)");
+}
+
 }  // namespace moe
 
 extern "C" int moe_debug_stall_next_tc_ffn(int calls) {
@@ -61,12 +95,21 @@ extern "C" int moe_debug_stall_next_tc_ffn(int calls) {
   return MOE_OK;
 }
 
+namespace moe {
+// The tensor-core path may run for this call (AUTO's choice, before any
+// fallback to the GEMV path on other hardware).
+static bool may_use_tc(int T, int k, int E, int path) {
+  if (path == MOE_PATH_TC) return true;
+  if (path == MOE_PATH_GEMV) return false;
+  return int64_t(T) * k >= int64_t(TC_MIN_ROWS_PER_EXPERT) * E;
+}
+}  // namespace moe
+
 extern "C" size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path) {
-  (void)E; (void)path;
-  if (T < 0 || k < 1 || I < 0) return moe::WS_HEADER;
-  // header | h [T*k][I] 16-bit | x as FP16 [T][H] (tensor-core path)
-  return moe::WS_HEADER + moe::round256(size_t(T) * size_t(k) * size_t(I) * 2) +
-         moe::round256(size_t(T) * size_t(H) * 2);
+  if (T < 0 || k < 1 || I < 0 || H < 0) return moe::WS_HEADER;
+  // header | h [T*k][I] 16-bit | x as FP16: [T][H] (GEMV) or [T*k][H] in group order (tensor cores)
+  const size_t xrows = moe::may_use_tc(T, k, E, path) ? size_t(T) * size_t(k) : size_t(T);
+  return moe::WS_HEADER + moe::round256(size_t(T) * size_t(k) * size_t(I) * 2) + moe::round256(xrows * size_t(H) * 2);
 }
 
 extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair, const int32_t *offsets,
@@ -111,14 +154,12 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
   a.h = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER);
   a.x16 = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER +
                                        round256(size_t(T) * size_t(k) * size_t(I) * 2));
+  a.xs = a.x16;
   a.y = y;
   a.stall = 0;
   if (T == 0) return MOE_OK;
 
-  int chosen = path;
-  if (path == MOE_PATH_AUTO)
-    chosen = (int64_t(T) * k >= int64_t(TC_MIN_ROWS_PER_EXPERT) * E) ? MOE_PATH_TC : MOE_PATH_GEMV;
-  if (chosen == MOE_PATH_TC) {
+  if (may_use_tc(T, k, E, path)) {
     a.stall = take_tc_stall();
     st = launch_ffn_tc(a, s);
     if (st != MOE_ERR_UNSUPPORTED || path == MOE_PATH_TC) return st;

@@ -18,7 +18,10 @@ struct FfnArgs {
   int64_t off_gq, off_uq, off_dq, off_gs, off_us, off_ds;  // record layout
   uint16_t *h;    // [P][I] workspace, sorted order: the BF16-rounded value
                   // stored as FP16 (exact), the down pass's B operand
-  uint16_t *x16;  // [T][H] FP16 copy of x, the gate/up pass's B operand
+  uint16_t *x16;  // [T][H] FP16 copy of x, the decode path's gate/up input
+  uint16_t *xs;   // [P][H] FP16 rows of x in group order (row r = token
+                  // sorted_pair[r] / k), the tensor-core gate/up B operand;
+                  // shares x16's workspace region
   float *y;       // [P][H] fp32 expert outputs, sorted order
   int32_t *err;   // device error word
   int stall;      // test hook: producers never publish a stage (bounded waits run out)
@@ -48,6 +51,7 @@ __device__ __forceinline__ uint4 ld_stream(const void *p) {
 }
 
 int launch_x_to_f16(const FfnArgs &a, cudaStream_t s);
+int launch_gather_x_f16(const FfnArgs &a, cudaStream_t s);
 int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s);
 int launch_ffn_tc(const FfnArgs &a, cudaStream_t s);
 

@@ -4,21 +4,30 @@
 // "Swap AB": the MMA's M dimension is 128 output features of one expert, its
 // N dimension is up to 256 of that expert's tokens (rows of the group, so a
 // small group runs a narrow MMA instead of a padded one), and K walks the
-// input features 64 at a time. N = 256 halves the shared-memory traffic per
-// FLOP of the dequantised A tile, which bounds this kernel. Per CTA (one per SM, persistent over a tile
-// list built on the device from the group offsets):
-//   warps 0-3  producers: gather the tile's token rows (cp.async, written in
-//              the 128-byte-swizzled K-major layout the MMA reads), copy the
-//              packed codes of their weight row, and dequantise them in
-//              registers to FP16 q*s straight into the swizzled A tile;
-//              fence.proxy.async, then arrive on `full`.
-//   warp 4     allocates tensor memory; one thread issues the MMAs
-//              (kind::f16 with FP16 A and B, fp32 accumulate) and commits each
-//              stage back to its `empty` barrier and each finished tile to
-//              `tmem_full`.
-//   warps 5-8  epilogue: tcgen05.ld of the accumulator (lane = feature,
-//              column = token), SwiGLU (gate/up pass) or the plain output
-//              (down pass), BF16 stores to h / y in group-sorted row order.
+// input features 64 at a time. Per CTA (one per SM, persistent over a tile
+// list built on the device from the group offsets), three rings of
+// shared-memory buffers, each k-step taking one slot of each:
+//   codes  the packed int4 codes of the tile's 128 weight rows (per matrix),
+//          small, so the ring runs 6-8 k-steps ahead of the MMA;
+//   B      256 FP16 activation rows (gate/up: x gathered into group order by
+//          a pre-pass; down: h), 128-byte-swizzled K-major as the MMA reads;
+//   A      the dequantised FP16 weights q*s, same swizzled layout.
+// Roles:
+//   warps 0-7   dequant: two threads per weight row read the codes from the
+//               codes ring (releasing the slot at once), wait for a free A
+//               slot, write FP16 q*s into it, fence.proxy.async, arrive.
+//   warps 8-15  epilogue: two warps per tensor-memory lane quadrant, each
+//               half of the token columns: tcgen05.ld of the accumulator
+//               (lane = feature, column = token), SwiGLU (gate/up pass) or the
+//               plain fp32 output (down pass), stores to h / y in group order.
+//   warp 16     allocates tensor memory; one thread issues the MMAs
+//               (kind::f16 with FP16 A and B, fp32 accumulate) and commits
+//               each k-step back to its A and B slots and each finished tile
+//               to `tmem_full`.
+//   warp 17     one thread issues the TMA loads of the codes ring (a 3-D box
+//               over the record bank: 32 bytes x 128 rows x 1 record).
+//   warp 18     one thread issues the TMA loads of the B ring (a 64 x 256
+//               FP16 box).
 // Why FP16 operands: q*s has at most 3 + 8 significant bits (|q| <= 8 and an
 // 8-bit BF16 scale significand) and FP16 holds 11, so the dequantised weight
 // is exact; a BF16 activation (8 significant bits) converts to FP16 exactly
@@ -31,8 +40,15 @@
 // FP16, which again is exact.
 // The down pass keeps two accumulator buffers so the epilogue of tile i
 // overlaps the mainloop of tile i+1; gate + up at N = 256 fill all 512
-// tensor-memory columns with one buffer. Every wait is bounded (about two seconds of %globaltimer); a wait
-// that runs out flags MOE_DEVERR_TIMEOUT and all roles drain and exit.
+// tensor-memory columns with one buffer, so there the epilogue is kept short
+// (eight warps, fast-divide SiLU) instead. Every wait is bounded (about two
+// seconds of %globaltimer); a wait that runs out flags MOE_DEVERR_TIMEOUT and
+// all roles drain and exit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "ffn.cuh"
 
 namespace moe {
@@ -40,26 +56,37 @@ namespace tc {
 
 constexpr int BM = 128;         // features per tile (MMA M)
 constexpr int BN = 256;         // max tokens per tile (MMA N)
-constexpr int BK = 64;          // K per stage (128 bytes of BF16 = one swizzle row)
-constexpr int MAX_STAGES = 5;
-constexpr int PRODUCERS = 256;  // warps 0-7: two threads per weight / token row of the tile
-constexpr int MMA_WARP = 8;
-constexpr int THREADS = 416;    // + warp 8 (MMA) + warps 9-12 (epilogue)
+constexpr int BK = 64;          // K per k-step (128 bytes of FP16 = one swizzle row)
+constexpr int MAX_RING = 8;
+constexpr int DEQUANT = 256;    // warps 0-7
+constexpr int EPI_WARP0 = 8;    // warps 8-15
+constexpr int EPILOGUE = 256;
+constexpr int MMA_WARP = 16;
+constexpr int TMA_CODES_WARP = 17;
+constexpr int TMA_B_WARP = 18;
+constexpr int THREADS = 608;
 constexpr uint64_t WAIT_NS = 2000000000ull;
 
 template <bool GATEUP>
 struct Cfg {
   static constexpr int NMAT = GATEUP ? 2 : 1;
-  static constexpr int A_BYTES = BM * BK * 2;         // 16 KB per matrix
+  static constexpr int A_BYTES = NMAT * BM * BK * 2;  // 16 KB per matrix
   static constexpr int B_BYTES = BN * BK * 2;         // 32 KB
-  static constexpr int NIB_BYTES = BM * 32 * NMAT;    // 32 bytes of codes per row and matrix
-  static constexpr int STAGE_BYTES = NMAT * A_BYTES + B_BYTES + NIB_BYTES;
-  static constexpr int STAGES = GATEUP ? 3 : 4;       // as many as fit in 227 KB
+  static constexpr int C_BYTES = NMAT * BM * BK / 2;  // 4 KB of codes per matrix
+  static constexpr int AS = GATEUP ? 2 : 3;           // ring depths
+  static constexpr int BS = GATEUP ? 3 : 4;
+  static constexpr int CS = GATEUP ? 6 : 8;
+  static constexpr int A_OFF = 0;
+  static constexpr int B_OFF = A_OFF + AS * A_BYTES;
+  static constexpr int C_OFF = B_OFF + BS * B_BYTES;
+  static constexpr int RING_BYTES = C_OFF + CS * C_BYTES;
   static constexpr int ACC_COLS = NMAT * BN;          // columns per accumulator buffer
   static constexpr int TMEM_COLS = 512;
   static constexpr int NBUF = TMEM_COLS / ACC_COLS;   // 1 (gate/up) or 2 (down) accumulator buffers
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 4096 /*tables, barriers*/;
+  static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 4096 /*tables, barriers*/;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(AS <= MAX_RING && BS <= MAX_RING && CS <= MAX_RING, "ring depth");
+  static_assert(B_OFF % 1024 == 0 && C_OFF % 1024 == 0, "swizzled buffers need 1024-byte alignment");
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -86,12 +113,24 @@ __device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// TMA tile loads (no multicast): completion counted in bytes on `bar`.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, int c0, int c1, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, int c0, int c1, int c2, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -135,7 +174,10 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 
 // ------------------------------------------------------------------ shared state
 struct Shared {
-  uint64_t full[MAX_STAGES], empty[MAX_STAGES], tmem_full[2], tmem_empty[2], drain;
+  uint64_t c_loaded[MAX_RING], c_free[MAX_RING];  // codes ring: TMA bytes / dequant threads
+  uint64_t b_loaded[MAX_RING], b_free[MAX_RING];  // B ring: TMA bytes / MMA commit
+  uint64_t a_full[MAX_RING], a_free[MAX_RING];    // A ring: dequant threads / MMA commit
+  uint64_t tmem_full[2], tmem_empty[2], drain;
   uint32_t tmem_base;
   int32_t abort;
   int32_t total_tiles;
@@ -184,27 +226,34 @@ __device__ __forceinline__ Tile decode_tile(const Shared &sh, int E, int FT, int
   return x;
 }
 
+// tm_b: activation rows in group order (gate/up: FP16 x gathered by the
+// pre-pass; down: h), box 64 x 256, 128-byte swizzle. tm_q0 / tm_q1: packed
+// codes of the first / second matrix over the record bank, box 32 B x 128
+// rows x 1 record.
 template <bool GATEUP>
-__global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_ffn_kernel(const FfnArgs a, const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_q0,
+                  const __grid_constant__ CUtensorMap tm_q1) {
   using C = Cfg<GATEUP>;
-  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Shared &sh = *reinterpret_cast<Shared *>(smem + STAGES * C::STAGE_BYTES);
+  Shared &sh = *reinterpret_cast<Shared *>(smem + C::RING_BYTES);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E;
   const int NOUT = GATEUP ? a.I : a.H;   // output features
   const int KD = GATEUP ? a.H : a.I;     // reduction length
   const int FT = NOUT / BM;              // feature tiles per token tile
-  const int KS = KD / BK;                // k-stages per tile
+  const int KS = KD / BK;                // k-steps per tile
   const int G = KD / GROUP;
   pdl_trigger();
   pdl_wait();
 
   // ---- prologue: barriers, tensor memory, tile table
   if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&sh.full[s], PRODUCERS); mbar_init(&sh.empty[s], 1); }
-    for (int b = 0; b < C::NBUF; ++b) { mbar_init(&sh.tmem_full[b], 1); mbar_init(&sh.tmem_empty[b], 128); }
+    for (int s = 0; s < C::CS; ++s) { mbar_init(&sh.c_loaded[s], 1); mbar_init(&sh.c_free[s], DEQUANT); }
+    for (int s = 0; s < C::BS; ++s) { mbar_init(&sh.b_loaded[s], 1); mbar_init(&sh.b_free[s], 1); }
+    for (int s = 0; s < C::AS; ++s) { mbar_init(&sh.a_full[s], DEQUANT); mbar_init(&sh.a_free[s], 1); }
+    for (int b = 0; b < C::NBUF; ++b) { mbar_init(&sh.tmem_full[b], 1); mbar_init(&sh.tmem_empty[b], EPILOGUE); }
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -253,123 +302,55 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
   const int total = sh.total_tiles;
   const int my_tiles = total > int(blockIdx.x) ? (total - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
   const int iters = my_tiles * KS;
-  auto stage_ptr = [&](int s) { return smem + s * C::STAGE_BYTES; };
+  uint8_t *const ringA = smem + C::A_OFF, *const ringB = smem + C::B_OFF, *const ringC = smem + C::C_OFF;
 
-  if (warp < PRODUCERS / 32) {
-    // ================================================================ producers
-    // Thread (p, i): i = row of the tile (weight row f0+i and token row i),
-    // p = which half of the row's work: the matrix (gate/up pass) or the K
-    // half of the stage (down pass), and half of the token row's 8 chunks.
+  if (warp < DEQUANT / 32) {
+    // ================================================================ dequant
+    // Thread (p, i): weight row f0+i of the tile; p = the matrix (gate/up
+    // pass) or the K half of the k-step (down pass).
     const int p = tid >> 7, i = tid & 127;
-    // per-tile state of the copy stream, refreshed when the stream enters a tile
-    int cur_tile = -1;
-    const uint8_t *qrow = nullptr;    // this thread's packed-code row
-    const uint16_t *srow = nullptr;   // its scale row
-    const uint16_t *brow_src[BN / BM] = {};
-    bool bvalid[BN / BM] = {};
-    auto enter_tile = [&](int tl_i) {
-      const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
-      const Tile tl = decode_tile(sh, E, FT, t);
-      const int slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
-      const uint8_t *rec = a.bank + int64_t(slot) * a.rec;
-      const int m = GATEUP ? p : 0;
-      qrow = rec + (GATEUP ? (m ? a.off_uq : a.off_gq) : a.off_dq) + int64_t(tl.f0 + i) * (KD / 2);
-      srow = reinterpret_cast<const uint16_t *>(rec + (GATEUP ? (m ? a.off_us : a.off_gs) : a.off_ds)) +
-             int64_t(tl.f0 + i) * G;
-#pragma unroll
-      for (int h = 0; h < BN / BM; ++h) {
-        const int r = i + h * BM;
-        bvalid[h] = r < tl.nvalid;
-        if (GATEUP) {
-          const int tok = bvalid[h] ? a.sorted_pair[tl.lo + tl.n0 + r] / a.k : 0;
-          brow_src[h] = a.x16 + int64_t(tok) * KD;
-        } else {
-          brow_src[h] = a.h + int64_t(bvalid[h] ? tl.lo + tl.n0 + r : 0) * KD;
-        }
-      }
-      cur_tile = tl_i;
-    };
-    // per-tile state of the dequant stream (lags the copies by D stages)
-    int deq_tile = -1;
+    int deq_tile = -1, ks = 0;
     const uint16_t *deq_srow = nullptr;
-    auto scale_row = [&](int tl_i) {
-      const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + tl_i * int(gridDim.x));
-      const int slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
-      const uint8_t *rec = a.bank + int64_t(slot) * a.rec;
-      const int m = GATEUP ? p : 0;
-      return reinterpret_cast<const uint16_t *>(rec + (GATEUP ? (m ? a.off_us : a.off_gs) : a.off_ds)) +
-             int64_t(tl.f0 + i) * G;
-    };
-    // Copies of stage `it` (cp.async); its group scale is prefetched into L1
-    // so the dequant D stages later reads it without a long stall.
-    auto issue = [&](int it) {
-      if (it / KS != cur_tile) enter_tile(it / KS);
-      const int ks = it % KS;
-      uint8_t *st = stage_ptr(it % STAGES);
-      const uint32_t nib = smem_u32(st + C::NMAT * C::A_BYTES + C::B_BYTES);
-      if (GATEUP) {  // matrix p: 32 bytes (64 codes) of row i; chunk c at slot c ^ ((i >> 2) & 1)
-        const uint32_t d = nib + (p * BM + i) * 32;
-        const int r = (i >> 2) & 1;
-        cp_async16(d + ((0 ^ r) << 4), qrow + ks * (BK / 2), 16);
-        cp_async16(d + ((1 ^ r) << 4), qrow + ks * (BK / 2) + 16, 16);
-      } else {       // K half p: 16 bytes (32 codes) of row i
-        cp_async16(nib + (i * 2 + p) * 16, qrow + ks * (BK / 2) + p * 16, 16);
-      }
-#pragma unroll
-      for (int h = 0; h < BN / BM; ++h) {  // token rows i and i + 128
-        const uint32_t brow = smem_u32(st + C::NMAT * C::A_BYTES) + (i + h * BM) * 128;
-#pragma unroll
-        for (int c = 4 * p; c < 4 * p + 4; ++c)
-          cp_async16(brow + ((c ^ (i & 7)) << 4), brow_src[h] + ks * BK + c * 8, bvalid[h] ? 16 : 0);
-      }
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(srow + (ks * BK) / GROUP));
-    };
-    constexpr int D = C::STAGES - 1;  // copy-ahead distance in stages
-    bool ok = true;
-#pragma unroll
-    for (int j = 0; j < D; ++j) {
-      if (j < iters && ok) {
-        ok = wait_bounded(sh, &sh.empty[j % STAGES], ((j / STAGES) & 1) ^ 1, a.err);
-        if (ok) issue(j);
-      }
-      cp_async_commit();
-    }
     const __half2 h1032 = __floats2half2_rn(1032.0f, 1032.0f);
     const __half2 h16th = __floats2half2_rn(0.0625f, 0.0625f);
     const __half2 hm72 = __floats2half2_rn(-72.0f, -72.0f);
-    // Per iteration: dequantise stage `it` and hand it to the MMA first, then
-    // refill the buffer the MMA has just finished with (stage it + D), so the
-    // dequant never waits for an MMA and the MMA finds each stage ready.
-    for (int it = 0; it < iters && ok; ++it) {
-      if (it / KS != deq_tile) { deq_tile = it / KS; deq_srow = scale_row(deq_tile); }
-      const uint16_t sbits = deq_srow[((it % KS) * BK) / GROUP];  // L1 hit (prefetched)
-      cp_async_wait<D - 1>();  // the copies of stage `it` have landed
-      // dequantise this thread's codes of stage `it` into the swizzled A tile
-      uint8_t *st = stage_ptr(it % STAGES);
-      const uint8_t *nib = st + C::NMAT * C::A_BYTES + C::B_BYTES;
-      const __half2 sc = __half2half2(__float2half_rn(bf16_to_f(sbits)));
+    bool ok = true;
+    for (int it = 0; it < iters && ok; ++it, ++ks) {
+      if (ks == KS || deq_tile < 0) {
+        ks = 0;
+        ++deq_tile;
+        const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + deq_tile * int(gridDim.x));
+        const int slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
+        const uint8_t *rec = a.bank + int64_t(slot) * a.rec;
+        deq_srow = reinterpret_cast<const uint16_t *>(rec + (GATEUP ? (p ? a.off_us : a.off_gs) : a.off_ds)) +
+                   int64_t(tl.f0 + i) * G;
+      }
+      const uint16_t sbits = deq_srow[(ks * BK) / GROUP];  // one 32-byte line per row and tile
+      const int cs = it % C::CS, as = it % C::AS;
+      ok = wait_bounded(sh, &sh.c_loaded[cs], (it / C::CS) & 1, a.err);
+      if (!ok) break;
+      const uint8_t *nib = ringC + cs * C::C_BYTES;  // [matrix][128 rows][32 B]
       uint32_t words[8];
-      int nw, c0;
-      uint8_t *arow;
       if (GATEUP) {
         const uint8_t *src = nib + (p * BM + i) * 32;
-        const int r = (i >> 2) & 1;
-        const uint4 w0 = *reinterpret_cast<const uint4 *>(src + ((0 ^ r) << 4));
-        const uint4 w1 = *reinterpret_cast<const uint4 *>(src + ((1 ^ r) << 4));
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(src);
+        const uint4 w1 = *reinterpret_cast<const uint4 *>(src + 16);
         words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
         words[4] = w1.x; words[5] = w1.y; words[6] = w1.z; words[7] = w1.w;
-        nw = 8; c0 = 0;
-        arow = st + p * C::A_BYTES + i * 128;
       } else {
-        const uint4 w0 = *reinterpret_cast<const uint4 *>(nib + (i * 2 + p) * 16);
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(nib + i * 32 + p * 16);
         words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
         words[4] = words[5] = words[6] = words[7] = 0;
-        nw = 4; c0 = 4 * p;
-        arow = st + i * 128;
       }
+      mbar_arrive(&sh.c_free[cs]);  // the codes are in registers: the slot may be refilled
+      ok = wait_bounded(sh, &sh.a_free[as], ((it / C::AS) & 1) ^ 1, a.err);
+      if (!ok) break;
+      const __half2 sc = __half2half2(__float2half_rn(bf16_to_f(sbits)));
+      constexpr int NW = GATEUP ? 8 : 4;
+      const int c0 = GATEUP ? 0 : 4 * p;
+      uint8_t *arow = ringA + as * C::A_BYTES + (GATEUP ? p * (BM * BK * 2) : 0) + i * 128;
 #pragma unroll
-      for (int wd = 0; wd < 8; ++wd) {
-        if (wd >= nw) break;
+      for (int wd = 0; wd < NW; ++wd) {
         // k = 2i + h sits at bits 4(i + 4h): OR-ing the nibbles at bits 0-3 /
         // 16-19 into FP16 1024.0 gives (1024 + u), those at bits 4-7 / 20-23
         // give (1024 + 16u); one shift by 8 brings pairs 2 and 3 to the same
@@ -389,15 +370,50 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
         *reinterpret_cast<uint4 *>(arow + ((c ^ (i & 7)) << 4)) = make_uint4(outp[0], outp[1], outp[2], outp[3]);
       }
       fence_proxy_async();
-      if (!a.stall) mbar_arrive(&sh.full[it % STAGES]);
-      const int nx = it + D;
-      if (nx < iters) {
-        ok = wait_bounded(sh, &sh.empty[nx % STAGES], ((nx / STAGES) & 1) ^ 1, a.err);
-        if (ok) issue(nx);
-      }
-      cp_async_commit();
+      if (!a.stall) mbar_arrive(&sh.a_full[as]);
     }
-    cp_async_wait<0>();
+  } else if (warp < EPI_WARP0 + EPILOGUE / 32) {
+    // ================================================================ epilogue
+    const int q = warp & 3;                          // tensor-memory lane quadrant of this warp
+    const int half = (warp - EPI_WARP0) >> 2;        // which half of the token columns
+    const int frow = q * 32 + lane;                  // feature within the tile
+    for (int tl_i = 0; tl_i < my_tiles; ++tl_i) {
+      const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
+      const Tile tl = decode_tile(sh, E, FT, t);
+      const int b = tl_i % C::NBUF;
+      if (!wait_bounded(sh, &sh.tmem_full[b], (tl_i / C::NBUF) & 1, a.err)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + (uint32_t(q * 32) << 16) + b * C::ACC_COLS;
+      const int f = tl.f0 + frow;
+      const int j_lo = half * (BN / 2), j_hi = min(tl.nvalid, j_lo + BN / 2);
+      const int64_t row0 = int64_t(tl.lo + tl.n0);
+      for (int j0 = j_lo; j0 < j_hi; j0 += 16) {
+        uint32_t g[16];
+        tmem_ld16(tbase + j0, g);
+        if (GATEUP) {
+          uint32_t u[16];
+          tmem_ld16(tbase + BN + j0, u);
+          tmem_wait_ld();
+          uint16_t *hp = a.h + (row0 + j0) * NOUT + f;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            if (j0 + jj < j_hi) {
+              const float gv = __uint_as_float(g[jj]), uv = __uint_as_float(u[jj]);
+              const float hv = bf16_to_f(f_to_bf16(silu_f(gv) * uv));  // A16: h is BF16
+              hp[jj * NOUT] = __half_as_ushort(__float2half_rn(hv));
+            }
+          }
+        } else {
+          tmem_wait_ld();
+          float *yp = a.y + (row0 + j0) * NOUT + f;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            if (j0 + jj < j_hi) yp[jj * NOUT] = __uint_as_float(g[jj]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sh.tmem_empty[b]);
+    }
   } else if (warp == MMA_WARP) {
     // ================================================================ MMA issuer
     if (lane == 0) {
@@ -414,20 +430,21 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
         tc_fence_after();
         const uint32_t d0 = tmem + b * C::ACC_COLS;
         for (int ks = 0; ks < KS; ++ks, ++it) {
-          const int s = it % STAGES;
-          ok = wait_bounded(sh, &sh.full[s], (it / STAGES) & 1, a.err);
+          const int as = it % C::AS, bs = it % C::BS;
+          ok = wait_bounded(sh, &sh.b_loaded[bs], (it / C::BS) & 1, a.err) &&
+               wait_bounded(sh, &sh.a_full[as], (it / C::AS) & 1, a.err);
           if (!ok) break;
           tc_fence_after();
-          uint8_t *st = stage_ptr(s);
-          const uint64_t bdesc = sw128_desc(smem_u32(st + C::NMAT * C::A_BYTES));
+          const uint64_t bdesc = sw128_desc(smem_u32(ringB + bs * C::B_BYTES));
 #pragma unroll
           for (int m = 0; m < C::NMAT; ++m) {
-            const uint64_t adesc = sw128_desc(smem_u32(st + m * C::A_BYTES));
+            const uint64_t adesc = sw128_desc(smem_u32(ringA + as * C::A_BYTES + m * (BM * BK * 2)));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
               mma_f16(d0 + m * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) != 0);
           }
-          mma_commit(&sh.empty[s]);
+          mma_commit(&sh.a_free[as]);
+          mma_commit(&sh.b_free[bs]);
         }
         if (ok) mma_commit(&sh.tmem_full[b]);
       }
@@ -436,46 +453,43 @@ __global__ void __launch_bounds__(THREADS, 1) tc_ffn_kernel(const FfnArgs a) {
       wait_bounded(sh, &sh.drain, 0, a.err, true);
     }
     __syncwarp();
-  } else {
-    // ================================================================ epilogue
-    const int q = warp & 3;            // tensor-memory lane quadrant of this warp
-    const int frow = q * 32 + lane;    // feature within the tile
-    for (int tl_i = 0; tl_i < my_tiles; ++tl_i) {
-      const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
-      const Tile tl = decode_tile(sh, E, FT, t);
-      const int b = tl_i % C::NBUF;
-      if (!wait_bounded(sh, &sh.tmem_full[b], (tl_i / C::NBUF) & 1, a.err)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem + (uint32_t(q * 32) << 16) + b * C::ACC_COLS;
-      const int f = tl.f0 + frow;
-      for (int j0 = 0; j0 < tl.nvalid; j0 += 16) {
-        uint32_t g[16];
-        tmem_ld16(tbase + j0, g);
-        if (GATEUP) {
-          uint32_t u[16];
-          tmem_ld16(tbase + BN + j0, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int j = j0 + jj;
-            if (j < tl.nvalid) {
-              const float gv = __uint_as_float(g[jj]), uv = __uint_as_float(u[jj]);
-              const float hv = bf16_to_f(f_to_bf16(silu_f(gv) * uv));  // A16: h is BF16
-              a.h[int64_t(tl.lo + tl.n0 + j) * NOUT + f] = __half_as_ushort(__float2half_rn(hv));
-            }
-          }
-        } else {
-          tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int j = j0 + jj;
-            if (j < tl.nvalid) a.y[int64_t(tl.lo + tl.n0 + j) * NOUT + f] = __uint_as_float(g[jj]);
-          }
+  } else if (warp == TMA_CODES_WARP || warp == TMA_B_WARP) {
+    // ================================================================ TMA
+    const bool codes = warp == TMA_CODES_WARP;
+    const int RING = codes ? C::CS : C::BS;
+    uint64_t *loaded = codes ? sh.c_loaded : sh.b_loaded;
+    uint64_t *freed = codes ? sh.c_free : sh.b_free;
+    if (lane == 0) {
+      int cur = -1, ks = 0, row_b = 0, f0 = 0, slot = 0, issued = 0;
+      bool ok = true;
+      for (int it = 0; it < iters && ok; ++it, ++ks) {
+        const int s = it % RING;
+        ok = wait_bounded(sh, &freed[s], ((it / RING) & 1) ^ 1, a.err);
+        if (!ok) break;
+        if (cur < 0 || ks == KS) {
+          ks = 0;
+          ++cur;
+          const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + cur * int(gridDim.x));
+          slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
+          row_b = tl.lo + tl.n0;  // first activation row of the tile, in group order
+          f0 = tl.f0;
         }
+        if (codes) {
+          uint8_t *dst = ringC + s * C::C_BYTES;
+          mbar_arrive_expect_tx(&loaded[s], C::C_BYTES);
+          tma_load_3d(dst, &tm_q0, ks * (BK / 2), f0, slot, &loaded[s]);
+          if (GATEUP) tma_load_3d(dst + BM * (BK / 2), &tm_q1, ks * (BK / 2), f0, slot, &loaded[s]);
+        } else {
+          mbar_arrive_expect_tx(&loaded[s], C::B_BYTES);
+          tma_load_2d(ringB + s * C::B_BYTES, &tm_b, ks * BK, row_b, &loaded[s]);
+        }
+        issued = it + 1;
       }
-      tc_fence_before();
-      mbar_arrive(&sh.tmem_empty[b]);
+      // every issued copy has landed before shared memory is released
+      for (int j = (issued > RING ? issued - RING : 0); j < issued; ++j)
+        wait_bounded(sh, &loaded[j % RING], (j / RING) & 1, a.err, true);
     }
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -501,6 +515,45 @@ static int sm_count() {
   return cached[dev];
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// FP16 rows [rows][cols] (cols contiguous), box 64 x 256 with the 128-byte
+// swizzle the MMA descriptors expect; rows past the end read as zero.
+static bool map_rows_f16(CUtensorMap *m, const void *base, int rows, int cols) {
+  const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  const cuuint32_t box[2] = {tc::BK, tc::BN};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed codes of one matrix in every record of the bank: bytes
+// [n_slots][nout][kd/2], box 32 bytes x 128 rows x 1 record, no swizzle.
+static bool map_codes(CUtensorMap *m, const uint8_t *bank, int64_t off, int64_t rec, int n_slots, int nout, int kd) {
+  const cuuint64_t dims[3] = {cuuint64_t(kd / 2), cuuint64_t(nout), cuuint64_t(n_slots)};
+  const cuuint64_t strides[2] = {cuuint64_t(kd / 2), cuuint64_t(rec)};
+  const cuuint32_t box[3] = {tc::BK / 2, tc::BM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(bank + off), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int launch_ffn_tc(const FfnArgs &a, cudaStream_t s) {
   int dev = 0, major = 0, minor = 0;
   cudaGetDevice(&dev);
@@ -511,19 +564,28 @@ int launch_ffn_tc(const FfnArgs &a, cudaStream_t s) {
                      minor);
   if (a.H % tc::BM || a.I % tc::BM)
     return set_error(MOE_ERR_UNSUPPORTED, "moe_grouped_w4a16_ffn: tensor-core path needs H, I multiples of 128");
+  if (!encode_fn())
+    return set_error(MOE_ERR_UNSUPPORTED, "moe_grouped_w4a16_ffn: cuTensorMapEncodeTiled is not available");
+  const int P = a.T * a.k;
+  CUtensorMap tm_xs, tm_h, tm_gq, tm_uq, tm_dq;
+  if (!map_rows_f16(&tm_xs, a.xs, P, a.H) || !map_rows_f16(&tm_h, a.h, P, a.I) ||
+      !map_codes(&tm_gq, a.bank, a.off_gq, a.rec, a.n_slots, a.I, a.H) ||
+      !map_codes(&tm_uq, a.bank, a.off_uq, a.rec, a.n_slots, a.I, a.H) ||
+      !map_codes(&tm_dq, a.bank, a.off_dq, a.rec, a.n_slots, a.H, a.I))
+    return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: tensor map encoding failed (pointers or strides)");
   const int grid = sm_count();
-  int st0 = launch_x_to_f16(a, s);
+  int st0 = launch_gather_x_f16(a, s);
   if (st0 != MOE_OK) return st0;
   const size_t smem_gu = tc::Cfg<true>::SMEM, smem_dn = tc::Cfg<false>::SMEM;
   int st = allow_dynamic_smem(reinterpret_cast<const void *>(tc::tc_ffn_kernel<true>), smem_gu, "ffn tc gate/up");
   if (st != MOE_OK) return st;
   st = allow_dynamic_smem(reinterpret_cast<const void *>(tc::tc_ffn_kernel<false>), smem_dn, "ffn tc down");
   if (st != MOE_OK) return st;
-  cudaError_t e = launch_pdl(tc::tc_ffn_kernel<true>, dim3(grid), dim3(tc::THREADS), smem_gu, s, a);
+  cudaError_t e = launch_pdl(tc::tc_ffn_kernel<true>, dim3(grid), dim3(tc::THREADS), smem_gu, s, a, tm_xs, tm_gq, tm_uq);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (tc gate/up): %s", cudaGetErrorString(e));
   st = check_launch("moe_grouped_w4a16_ffn (tc gate/up)");
   if (st != MOE_OK) return st;
-  e = launch_pdl(tc::tc_ffn_kernel<false>, dim3(grid), dim3(tc::THREADS), smem_dn, s, a);
+  e = launch_pdl(tc::tc_ffn_kernel<false>, dim3(grid), dim3(tc::THREADS), smem_dn, s, a, tm_h, tm_dq, tm_dq);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (tc down): %s", cudaGetErrorString(e));
   return check_launch("moe_grouped_w4a16_ffn (tc down)");
 }
