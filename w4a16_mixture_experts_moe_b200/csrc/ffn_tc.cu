@@ -73,19 +73,18 @@ struct Cfg {
   static constexpr int A_BYTES = NMAT * BM * BK * 2;  // 16 KB per matrix
   static constexpr int B_BYTES = BN * BK * 2;         // 32 KB
   static constexpr int C_BYTES = NMAT * BM * BK / 2;  // 4 KB of codes per matrix
-  static constexpr int AS = GATEUP ? 2 : 3;           // ring depths
-  static constexpr int BS = GATEUP ? 3 : 4;
-  static constexpr int CS = GATEUP ? 6 : 8;
+  static constexpr int S = GATEUP ? 3 : 4;            // A and B ring depth (one commit frees both)
+  static constexpr int CS = GATEUP ? 3 : 4;           // codes ring depth
   static constexpr int A_OFF = 0;
-  static constexpr int B_OFF = A_OFF + AS * A_BYTES;
-  static constexpr int C_OFF = B_OFF + BS * B_BYTES;
+  static constexpr int B_OFF = A_OFF + S * A_BYTES;
+  static constexpr int C_OFF = B_OFF + S * B_BYTES;
   static constexpr int RING_BYTES = C_OFF + CS * C_BYTES;
   static constexpr int ACC_COLS = NMAT * BN;          // columns per accumulator buffer
   static constexpr int TMEM_COLS = 512;
   static constexpr int NBUF = TMEM_COLS / ACC_COLS;   // 1 (gate/up) or 2 (down) accumulator buffers
   static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 4096 /*tables, barriers*/;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
-  static_assert(AS <= MAX_RING && BS <= MAX_RING && CS <= MAX_RING, "ring depth");
+  static_assert(S <= MAX_RING && CS <= MAX_RING, "ring depth");
   static_assert(B_OFF % 1024 == 0 && C_OFF % 1024 == 0, "swizzled buffers need 1024-byte alignment");
 };
 
@@ -131,6 +130,16 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, in
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
+// One lane of a converged warp (the lowest), chosen by elect.sync: the
+// issue idiom for tcgen05 and TMA instructions, whose operands then stay in
+// uniform registers.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n .reg .b32 r;\n .reg .pred p;\n elect.sync r|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -175,8 +184,8 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // ------------------------------------------------------------------ shared state
 struct Shared {
   uint64_t c_loaded[MAX_RING], c_free[MAX_RING];  // codes ring: TMA bytes / dequant threads
-  uint64_t b_loaded[MAX_RING], b_free[MAX_RING];  // B ring: TMA bytes / MMA commit
-  uint64_t a_full[MAX_RING], a_free[MAX_RING];    // A ring: dequant threads / MMA commit
+  uint64_t b_loaded[MAX_RING], a_full[MAX_RING];  // stage s: B rows landed (TMA bytes) / A written (dequant warps)
+  uint64_t s_free[MAX_RING];                      // stage s: its MMAs completed (commit)
   uint64_t tmem_full[2], tmem_empty[2], drain;
   uint32_t tmem_base;
   int32_t abort;
@@ -191,13 +200,17 @@ struct Shared {
 // MMAs still in flight).
 __device__ __noinline__ bool wait_bounded(Shared &sh, uint64_t *bar, uint32_t parity, int32_t *err,
                                           bool drain = false) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  // %globaltimer is read only every 256 polls (the first time after 256): a
+  // wait that ends soon never pays for the timer read.
+  uint64_t t0 = 0;
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try(bar, parity)) return true;
     if ((spin & 255) == 0) {
       if (!drain && *(volatile int32_t *)&sh.abort) return false;
-      if (globaltimer() - t0 > WAIT_NS) {
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > WAIT_NS) {
         atomicExch(&sh.abort, 1);
         flag_error(err, MOE_DEVERR_TIMEOUT);
         return false;
@@ -250,10 +263,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // ---- prologue: barriers, tensor memory, tile table
   if (tid == 0) {
-    for (int s = 0; s < C::CS; ++s) { mbar_init(&sh.c_loaded[s], 1); mbar_init(&sh.c_free[s], DEQUANT); }
-    for (int s = 0; s < C::BS; ++s) { mbar_init(&sh.b_loaded[s], 1); mbar_init(&sh.b_free[s], 1); }
-    for (int s = 0; s < C::AS; ++s) { mbar_init(&sh.a_full[s], DEQUANT); mbar_init(&sh.a_free[s], 1); }
-    for (int b = 0; b < C::NBUF; ++b) { mbar_init(&sh.tmem_full[b], 1); mbar_init(&sh.tmem_empty[b], EPILOGUE); }
+    // consumer-side barriers count one elected arrival per warp
+    for (int s = 0; s < C::CS; ++s) { mbar_init(&sh.c_loaded[s], 1); mbar_init(&sh.c_free[s], DEQUANT / 32); }
+    for (int s = 0; s < C::S; ++s) {
+      mbar_init(&sh.b_loaded[s], 1);
+      mbar_init(&sh.a_full[s], DEQUANT / 32);
+      mbar_init(&sh.s_free[s], 1);
+    }
+    for (int b = 0; b < C::NBUF; ++b) { mbar_init(&sh.tmem_full[b], 1); mbar_init(&sh.tmem_empty[b], EPILOGUE / 32); }
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -326,8 +343,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                    int64_t(tl.f0 + i) * G;
       }
       const uint16_t sbits = deq_srow[(ks * BK) / GROUP];  // one 32-byte line per row and tile
-      const int cs = it % C::CS, as = it % C::AS;
-      ok = wait_bounded(sh, &sh.c_loaded[cs], (it / C::CS) & 1, a.err);
+      const int cs = it % C::CS, as = it % C::S;
+      // wait results are made warp-uniform: a lane never leaves the loop
+      // while the rest of its warp goes on to a __syncwarp
+      ok = __all_sync(0xffffffffu, wait_bounded(sh, &sh.c_loaded[cs], (it / C::CS) & 1, a.err));
       if (!ok) break;
       const uint8_t *nib = ringC + cs * C::C_BYTES;  // [matrix][128 rows][32 B]
       uint32_t words[8];
@@ -342,8 +361,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
         words[4] = words[5] = words[6] = words[7] = 0;
       }
-      mbar_arrive(&sh.c_free[cs]);  // the codes are in registers: the slot may be refilled
-      ok = wait_bounded(sh, &sh.a_free[as], ((it / C::AS) & 1) ^ 1, a.err);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.c_free[cs]);  // the warp's codes are in registers: the slot may be refilled
+      ok = __all_sync(0xffffffffu, wait_bounded(sh, &sh.s_free[as], ((it / C::S) & 1) ^ 1, a.err));
       if (!ok) break;
       const __half2 sc = __half2half2(__float2half_rn(bf16_to_f(sbits)));
       constexpr int NW = GATEUP ? 8 : 4;
@@ -369,8 +389,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int c = c0 + wd;
         *reinterpret_cast<uint4 *>(arow + ((c ^ (i & 7)) << 4)) = make_uint4(outp[0], outp[1], outp[2], outp[3]);
       }
-      fence_proxy_async();
-      if (!a.stall) mbar_arrive(&sh.a_full[as]);
+      fence_proxy_async();  // this thread's A writes -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0 && !a.stall) mbar_arrive(&sh.a_full[as]);
     }
   } else if (warp < EPI_WARP0 + EPILOGUE / 32) {
     // ================================================================ epilogue
@@ -381,7 +402,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
       const Tile tl = decode_tile(sh, E, FT, t);
       const int b = tl_i % C::NBUF;
-      if (!wait_bounded(sh, &sh.tmem_full[b], (tl_i / C::NBUF) & 1, a.err)) break;
+      if (!__all_sync(0xffffffffu, wait_bounded(sh, &sh.tmem_full[b], (tl_i / C::NBUF) & 1, a.err))) break;
       tc_fence_after();
       const uint32_t tbase = tmem + (uint32_t(q * 32) << 16) + b * C::ACC_COLS;
       const int f = tl.f0 + frow;
@@ -412,68 +433,96 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&sh.tmem_empty[b]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.tmem_empty[b]);
     }
   } else if (warp == MMA_WARP) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      for (int tl_i = 0; tl_i < my_tiles && ok; ++tl_i) {
-        const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
-        const Tile tl = decode_tile(sh, E, FT, t);
-        const int n_mma = max(16, (tl.nvalid + 15) & ~15);
-        const uint32_t idesc = idesc_f16(n_mma);
-        const int b = tl_i % C::NBUF;
-        ok = wait_bounded(sh, &sh.tmem_empty[b], ((tl_i / C::NBUF) & 1) ^ 1, a.err);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t d0 = tmem + b * C::ACC_COLS;
-        for (int ks = 0; ks < KS; ++ks, ++it) {
-          const int as = it % C::AS, bs = it % C::BS;
-          ok = wait_bounded(sh, &sh.b_loaded[bs], (it / C::BS) & 1, a.err) &&
-               wait_bounded(sh, &sh.a_full[as], (it / C::AS) & 1, a.err);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t bdesc = sw128_desc(smem_u32(ringB + bs * C::B_BYTES));
+    // The whole warp runs the loop and every lane waits (results made
+    // warp-uniform); one elected lane issues the MMAs and the commits, so
+    // descriptors are computed converged. Everything needed to issue k-step
+    // it+1 is waited for before k-step it is committed, so the tensor core's
+    // queue is refilled without a commit in between (and between tiles when
+    // there are two accumulator buffers; with one, the next tile waits for
+    // the epilogue anyway).
+    bool ok = true;
+    auto ready = [&](int it) {  // stage it % S: B rows landed and A tile written
+      const int s = it % C::S;
+      const bool r = wait_bounded(sh, &sh.b_loaded[s], (it / C::S) & 1, a.err) &&
+                     wait_bounded(sh, &sh.a_full[s], (it / C::S) & 1, a.err);
+      return __all_sync(0xffffffffu, r);
+    };
+    auto acc_free = [&](int tl_i) {  // the tile's accumulator buffer was drained by the epilogue
+      const bool r = wait_bounded(sh, &sh.tmem_empty[tl_i % C::NBUF], ((tl_i / C::NBUF) & 1) ^ 1, a.err);
+      return __all_sync(0xffffffffu, r);
+    };
+    if (iters > 0) ok = acc_free(0) && ready(0);
+    int tl_i = 0, ks = 0;
+    Tile tl = decode_tile(sh, E, FT, int(blockIdx.x));
+    for (int it = 0; it < iters && ok; ++it) {
+      tc_fence_after();
+      const int s = it % C::S, b = tl_i % C::NBUF;
+      const uint32_t idesc = idesc_f16(max(16, (tl.nvalid + 15) & ~15));
+      const uint32_t d0 = tmem + b * C::ACC_COLS;
+      const uint64_t bdesc = sw128_desc(smem_u32(ringB + s * C::B_BYTES));
+      const uint64_t adesc0 = sw128_desc(smem_u32(ringA + s * C::A_BYTES));
+      if (elect_one()) {
 #pragma unroll
-          for (int m = 0; m < C::NMAT; ++m) {
-            const uint64_t adesc = sw128_desc(smem_u32(ringA + as * C::A_BYTES + m * (BM * BK * 2)));
+        for (int m = 0; m < C::NMAT; ++m) {
+          const uint64_t adesc = adesc0 + uint64_t((m * (BM * BK * 2)) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              mma_f16(d0 + m * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) != 0);
-          }
-          mma_commit(&sh.a_free[as]);
-          mma_commit(&sh.b_free[bs]);
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_f16(d0 + m * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) != 0);
         }
-        if (ok) mma_commit(&sh.tmem_full[b]);
       }
-      // all issued MMAs have completed before tensor memory is released
-      mma_commit(&sh.drain);
-      wait_bounded(sh, &sh.drain, 0, a.err, true);
+      __syncwarp();
+      const bool has_next = it + 1 < iters;
+      if (ks + 1 < KS) {
+        ok = ready(it + 1);
+        if (elect_one()) mma_commit(&sh.s_free[s]);
+        ++ks;
+      } else {
+        if (C::NBUF > 1 && has_next) {
+          ok = acc_free(tl_i + 1) && ready(it + 1);
+          if (elect_one()) { mma_commit(&sh.s_free[s]); mma_commit(&sh.tmem_full[b]); }
+        } else {
+          if (elect_one()) { mma_commit(&sh.s_free[s]); mma_commit(&sh.tmem_full[b]); }
+          __syncwarp();
+          if (has_next) ok = acc_free(tl_i + 1) && ready(it + 1);
+        }
+        ks = 0;
+        ++tl_i;
+        if (has_next) tl = decode_tile(sh, E, FT, int(blockIdx.x) + tl_i * int(gridDim.x));
+      }
+      __syncwarp();
     }
+    // all issued MMAs have completed before tensor memory is released
+    if (elect_one()) mma_commit(&sh.drain);
+    __syncwarp();
+    wait_bounded(sh, &sh.drain, 0, a.err, true);
     __syncwarp();
   } else if (warp == TMA_CODES_WARP || warp == TMA_B_WARP) {
     // ================================================================ TMA
+    // converged warp; every lane waits, one elected lane issues
     const bool codes = warp == TMA_CODES_WARP;
-    const int RING = codes ? C::CS : C::BS;
+    const int RING = codes ? C::CS : C::S;
     uint64_t *loaded = codes ? sh.c_loaded : sh.b_loaded;
-    uint64_t *freed = codes ? sh.c_free : sh.b_free;
-    if (lane == 0) {
-      int cur = -1, ks = 0, row_b = 0, f0 = 0, slot = 0, issued = 0;
-      bool ok = true;
-      for (int it = 0; it < iters && ok; ++it, ++ks) {
-        const int s = it % RING;
-        ok = wait_bounded(sh, &freed[s], ((it / RING) & 1) ^ 1, a.err);
-        if (!ok) break;
-        if (cur < 0 || ks == KS) {
-          ks = 0;
-          ++cur;
-          const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + cur * int(gridDim.x));
-          slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
-          row_b = tl.lo + tl.n0;  // first activation row of the tile, in group order
-          f0 = tl.f0;
-        }
+    uint64_t *freed = codes ? sh.c_free : sh.s_free;
+    int cur = -1, ks = 0, row_b = 0, f0 = 0, slot = 0, issued = 0;
+    bool ok = true;
+    for (int it = 0; it < iters && ok; ++it, ++ks) {
+      const int s = it % RING;
+      ok = __all_sync(0xffffffffu, wait_bounded(sh, &freed[s], ((it / RING) & 1) ^ 1, a.err));
+      if (!ok) break;
+      if (cur < 0 || ks == KS) {
+        ks = 0;
+        ++cur;
+        const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + cur * int(gridDim.x));
+        slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
+        row_b = tl.lo + tl.n0;  // first activation row of the tile, in group order
+        f0 = tl.f0;
+      }
+      if (elect_one()) {
         if (codes) {
           uint8_t *dst = ringC + s * C::C_BYTES;
           mbar_arrive_expect_tx(&loaded[s], C::C_BYTES);
@@ -483,12 +532,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_arrive_expect_tx(&loaded[s], C::B_BYTES);
           tma_load_2d(ringB + s * C::B_BYTES, &tm_b, ks * BK, row_b, &loaded[s]);
         }
-        issued = it + 1;
       }
-      // every issued copy has landed before shared memory is released
-      for (int j = (issued > RING ? issued - RING : 0); j < issued; ++j)
-        wait_bounded(sh, &loaded[j % RING], (j / RING) & 1, a.err, true);
+      __syncwarp();
+      issued = it + 1;
     }
+    // every issued copy has landed before shared memory is released
+    for (int j = (issued > RING ? issued - RING : 0); j < issued; ++j)
+      wait_bounded(sh, &loaded[j % RING], (j / RING) & 1, a.err, true);
     __syncwarp();
   }
 
