@@ -20,10 +20,17 @@
 //               half of the token columns: tcgen05.ld of the accumulator
 //               (lane = feature, column = token), SwiGLU (gate/up pass) or the
 //               plain fp32 output (down pass), stores to h / y in group order.
-//   warp 16     allocates tensor memory; one thread issues the MMAs
+//   warp 16     allocates tensor memory; one elected lane issues the MMAs
 //               (kind::f16 with FP16 A and B, fp32 accumulate) and commits
 //               each k-step back to its A and B slots and each finished tile
-//               to `tmem_full`.
+//               to `tmem_full`. It touches no memory inside the loop: a
+//               warp's loads, stores and mbarrier waits issued behind
+//               tcgen05.mma are held until those MMAs finish, which would
+//               drain the tensor core's short queue at every k-step.
+//   warp 19     waiter: performs the bounded mbarrier waits for the MMA warp
+//               (stage landed and dequantised, accumulator buffer free) and
+//               hands each k-step over with a named-barrier reduction
+//               (bar.red.popc) carrying the tile's MMA width and an abort bit.
 //   warp 17     one thread issues the TMA loads of the codes ring (a 3-D box
 //               over the record bank: 32 bytes x 128 rows x 1 record).
 //   warp 18     one thread issues the TMA loads of the B ring (a 64 x 256
@@ -64,7 +71,9 @@ constexpr int EPILOGUE = 256;
 constexpr int MMA_WARP = 16;
 constexpr int TMA_CODES_WARP = 17;
 constexpr int TMA_B_WARP = 18;
-constexpr int THREADS = 608;
+constexpr int WAITER_WARP = 19;
+constexpr int THREADS = 640;
+constexpr int HANDOFF_BAR = 1;  // named barrier: waiter warp + MMA warp
 constexpr uint64_t WAIT_NS = 2000000000ull;
 
 template <bool GATEUP>
@@ -139,6 +148,16 @@ __device__ __forceinline__ bool elect_one() {
       "{\n .reg .b32 r;\n .reg .pred p;\n elect.sync r|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(pred));
   return pred != 0;
+}
+// Named-barrier handoff between the waiter and the MMA warp (64 threads):
+// returns the number of participating threads whose predicate is true.
+__device__ __forceinline__ uint32_t handoff(uint32_t pred) {
+  uint32_t cnt;
+  asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n bar.red.popc.u32 %0, %2, 64, p;\n}\n"
+               : "=r"(cnt)
+               : "r"(pred), "n"(HANDOFF_BAR)
+               : "memory");
+  return cnt;
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -438,31 +457,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == MMA_WARP) {
     // ================================================================ MMA issuer
-    // The whole warp runs the loop and every lane waits (results made
-    // warp-uniform); one elected lane issues the MMAs and the commits, so
-    // descriptors are computed converged. Everything needed to issue k-step
-    // it+1 is waited for before k-step it is committed, so the tensor core's
-    // queue is refilled without a commit in between (and between tiles when
-    // there are two accumulator buffers; with one, the next tile waits for
-    // the epilogue anyway).
-    bool ok = true;
-    auto ready = [&](int it) {  // stage it % S: B rows landed and A tile written
-      const int s = it % C::S;
-      const bool r = wait_bounded(sh, &sh.b_loaded[s], (it / C::S) & 1, a.err) &&
-                     wait_bounded(sh, &sh.a_full[s], (it / C::S) & 1, a.err);
-      return __all_sync(0xffffffffu, r);
-    };
-    auto acc_free = [&](int tl_i) {  // the tile's accumulator buffer was drained by the epilogue
-      const bool r = wait_bounded(sh, &sh.tmem_empty[tl_i % C::NBUF], ((tl_i / C::NBUF) & 1) ^ 1, a.err);
-      return __all_sync(0xffffffffu, r);
-    };
-    if (iters > 0) ok = acc_free(0) && ready(0);
-    int tl_i = 0, ks = 0;
-    Tile tl = decode_tile(sh, E, FT, int(blockIdx.x));
-    for (int it = 0; it < iters && ok; ++it) {
+    // Per k-step: one handoff from the waiter (count = n16 = MMA width / 16,
+    // 1..16, or > 16 to stop), then the MMAs and commits from one elected
+    // lane. Tile boundaries are found by counting k-steps.
+    int ks = 0, tl_i = 0;
+    for (int it = 0; it < iters; ++it) {
+      const uint32_t v = handoff(0);
+      if (v > 16) break;
       tc_fence_after();
       const int s = it % C::S, b = tl_i % C::NBUF;
-      const uint32_t idesc = idesc_f16(max(16, (tl.nvalid + 15) & ~15));
+      const uint32_t idesc = idesc_f16(int(v) * 16);
       const uint32_t d0 = tmem + b * C::ACC_COLS;
       const uint64_t bdesc = sw128_desc(smem_u32(ringB + s * C::B_BYTES));
       const uint64_t adesc0 = sw128_desc(smem_u32(ringA + s * C::A_BYTES));
@@ -474,33 +478,40 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int kk = 0; kk < BK / 16; ++kk)
             mma_f16(d0 + m * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) != 0);
         }
+        mma_commit(&sh.s_free[s]);
+        if (ks + 1 == KS) mma_commit(&sh.tmem_full[b]);
       }
       __syncwarp();
-      const bool has_next = it + 1 < iters;
-      if (ks + 1 < KS) {
-        ok = ready(it + 1);
-        if (elect_one()) mma_commit(&sh.s_free[s]);
-        ++ks;
-      } else {
-        if (C::NBUF > 1 && has_next) {
-          ok = acc_free(tl_i + 1) && ready(it + 1);
-          if (elect_one()) { mma_commit(&sh.s_free[s]); mma_commit(&sh.tmem_full[b]); }
-        } else {
-          if (elect_one()) { mma_commit(&sh.s_free[s]); mma_commit(&sh.tmem_full[b]); }
-          __syncwarp();
-          if (has_next) ok = acc_free(tl_i + 1) && ready(it + 1);
-        }
-        ks = 0;
-        ++tl_i;
-        if (has_next) tl = decode_tile(sh, E, FT, int(blockIdx.x) + tl_i * int(gridDim.x));
-      }
-      __syncwarp();
+      if (++ks == KS) { ks = 0; ++tl_i; }
     }
     // all issued MMAs have completed before tensor memory is released
     if (elect_one()) mma_commit(&sh.drain);
     __syncwarp();
     wait_bounded(sh, &sh.drain, 0, a.err, true);
     __syncwarp();
+  } else if (warp == WAITER_WARP) {
+    // ================================================================ waiter
+    // For each k-step of the MMA warp: (at a tile's first k-step) its
+    // accumulator buffer has been drained by the epilogue, then the stage's
+    // B rows have landed and its A tile is written; every wait bounded. The
+    // handoff carries n16 = MMA width / 16 (lanes below n16 vote), plus 16
+    // votes (lanes 16-31) when a wait failed, after which both warps stop.
+    int ks = 0, tl_i = 0, n16 = 1;
+    for (int it = 0; it < iters; ++it) {
+      bool ok = true;
+      if (ks == 0) {
+        const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + tl_i * int(gridDim.x));
+        n16 = max(1, (tl.nvalid + 15) >> 4);
+        ok = wait_bounded(sh, &sh.tmem_empty[tl_i % C::NBUF], ((tl_i / C::NBUF) & 1) ^ 1, a.err);
+      }
+      const int s = it % C::S;
+      ok = ok && wait_bounded(sh, &sh.b_loaded[s], (it / C::S) & 1, a.err) &&
+           wait_bounded(sh, &sh.a_full[s], (it / C::S) & 1, a.err);
+      ok = __all_sync(0xffffffffu, ok);
+      handoff(lane < n16 || (!ok && lane >= 16));
+      if (!ok) break;
+      if (++ks == KS) { ks = 0; ++tl_i; }
+    }
   } else if (warp == TMA_CODES_WARP || warp == TMA_B_WARP) {
     // ================================================================ TMA
     // converged warp; every lane waits, one elected lane issues
