@@ -41,15 +41,6 @@ __device__ __forceinline__ const uint8_t *expert_record(const FfnArgs &a, int e)
   return a.bank + int64_t(slot) * a.rec;
 }
 
-// Streaming 16-byte load that skips L1 (weights are read once).
-__device__ __forceinline__ uint4 ld_stream(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 int launch_x_to_f16(const FfnArgs &a, cudaStream_t s);
 int launch_gather_x_f16(const FfnArgs &a, cudaStream_t s);
 int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s);

@@ -15,6 +15,13 @@
 // group is then multiplied by that row's group scale, so the dequantised
 // weight q*s is never rounded.
 //
+// The codes stream through a per-warp shared-memory ring of GV_DEPTH group
+// slots filled by cp.async, GV_DEPTH - 1 groups ahead of the math: the bytes
+// in flight per SM then do not depend on registers, and at the loaded HBM
+// latency they are what bounds a streaming kernel's bandwidth. Each lane
+// copies, and later reads back, only its own 16-byte pieces, so its own
+// cp.async waits suffice.
+//
 // Why FP16 operands: this kernel is bound by integer instructions spent
 // unpacking codes, and FP16's 10-bit mantissa lets a nibble sit at bits 4-7
 // of a half: one LOP3 yields (1024 + u) and another (1024 + 16u) for the next
@@ -27,7 +34,17 @@
 namespace moe {
 
 constexpr int GV_WARPS = 4;  // 64 rows per CTA
-constexpr int GV_UNROLL = 4;
+constexpr int GV_DEPTH = 4;  // groups of codes in flight per warp (shared-memory ring)
+
+// 16-byte asynchronous copy global -> shared, cached in L2 only.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -93,6 +110,7 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint4 &w0, cons
 template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArgs a) {
   __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][8][32];
+  __shared__ uint4 rings[GV_WARPS][GV_DEPTH * 4 * 32];  // [slot][gate g, gate g+8, up g, up g+8][lane]
   pdl_trigger();
   pdl_wait();
   const int e = blockIdx.y;
@@ -117,10 +135,28 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
     const int token = ok ? a.sorted_pair[lo + n0 + g] / a.k : 0;
     const uint16_t *xr = a.x16 + int64_t(token) * H + t * 32;
     float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll GV_UNROLL
-    for (int grp = kq; grp < (rows_ok ? G : 0); grp += KS) {
-      const uint4 g0 = ld_stream(gq0 + grp * 64), g1 = ld_stream(gq0 + 8 * KB + grp * 64);
-      const uint4 u0 = ld_stream(uq0 + grp * 64), u1 = ld_stream(uq0 + 8 * KB + grp * 64);
+    const int ngrp = rows_ok && kq < G ? (G - 1 - kq) / KS + 1 : 0;
+    uint4 *ring = rings[warp];
+    auto issue = [&](int i) {
+      const int grp = kq + i * KS;
+      uint4 *d = ring + (i % GV_DEPTH) * (4 * 32) + lane;
+      cp_async16(d, gq0 + grp * 64);
+      cp_async16(d + 32, gq0 + 8 * KB + grp * 64);
+      cp_async16(d + 64, uq0 + grp * 64);
+      cp_async16(d + 96, uq0 + 8 * KB + grp * 64);
+    };
+#pragma unroll
+    for (int i = 0; i < GV_DEPTH - 1; ++i) {
+      if (i < ngrp) issue(i);
+      cp_async_commit();
+    }
+    for (int i = 0; i < ngrp; ++i) {
+      const int grp = kq + i * KS;
+      if (i + GV_DEPTH - 1 < ngrp) issue(i + GV_DEPTH - 1);
+      cp_async_commit();
+      cp_async_wait<GV_DEPTH - 1>();  // group i's copies (this lane's) have landed
+      const uint4 *sr = ring + (i % GV_DEPTH) * (4 * 32) + lane;
+      const uint4 g0 = sr[0], g1 = sr[32], u0 = sr[64], u1 = sr[96];
       uint4 xb[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -167,6 +203,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
 template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs a) {
   __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][4][32];
+  __shared__ uint4 rings[GV_WARPS][GV_DEPTH * 2 * 32];  // [slot][row g, row g+8][lane]
   pdl_trigger();
   pdl_wait();
   const int e = blockIdx.y;
@@ -188,9 +225,26 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
     const bool ok = n0 + g < cnt;
     const uint16_t *hr = a.h + int64_t(lo + (ok ? n0 + g : 0)) * I + t * 32;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll GV_UNROLL
-    for (int grp = kq; grp < (rows_ok ? G : 0); grp += KS) {
-      const uint4 w0 = ld_stream(dq0 + grp * 64), w1 = ld_stream(dq0 + 8 * KB + grp * 64);
+    const int ngrp = rows_ok && kq < G ? (G - 1 - kq) / KS + 1 : 0;
+    uint4 *ring = rings[warp];
+    auto issue = [&](int i) {
+      const int grp = kq + i * KS;
+      uint4 *d = ring + (i % GV_DEPTH) * (2 * 32) + lane;
+      cp_async16(d, dq0 + grp * 64);
+      cp_async16(d + 32, dq0 + 8 * KB + grp * 64);
+    };
+#pragma unroll
+    for (int i = 0; i < GV_DEPTH - 1; ++i) {
+      if (i < ngrp) issue(i);
+      cp_async_commit();
+    }
+    for (int i = 0; i < ngrp; ++i) {
+      const int grp = kq + i * KS;
+      if (i + GV_DEPTH - 1 < ngrp) issue(i + GV_DEPTH - 1);
+      cp_async_commit();
+      cp_async_wait<GV_DEPTH - 1>();  // group i's copies (this lane's) have landed
+      const uint4 *sr = ring + (i % GV_DEPTH) * (2 * 32) + lane;
+      const uint4 w0 = sr[0], w1 = sr[32];
       uint4 xb[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q)
