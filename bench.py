@@ -38,6 +38,13 @@ SWEEP_T = (1, 4, 16, 64)
 METRIC = "MoE-layer tokens/s; HBM GB/s (decode) and TC TFLOP/s (prefill) vs B200 peak"
 SHAPES = {"olmoe": (2048, 1024, 64, 8), "wide": (4096, 14336, 8, 2)}   # (H, I, E, k)
 
+# DRAM bytes (read + write) of one decode FFN call per active expert, from one
+# ncu capture of the gate/up and down GEMV launches at T=16 (57 active
+# experts: 123.60 MB + 60.24 MB).
+# Reported as roofline.traffic scaled to the bench's active experts; valid
+# while those kernels are the ones captured.
+DECODE_TRAFFIC_PER_ACTIVE_EXPERT = (123.600e6 + 60.236e6) / 57
+
 
 def rec_bytes(h, i):
     """Bytes of one packed expert record: codes of three matrices + their scales."""
@@ -389,7 +396,10 @@ def main():
                     "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
             "roofline": {"bound": "hbm", "kernel": "moe_grouped_w4a16_ffn (gate/up + down kernels), per layer call",
                          "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / P["hbm_gbs"], "traffic": None,
+                         "frac": achieved / P["hbm_gbs"],
+                         "traffic": (DECODE_TRAFFIC_PER_ACTIVE_EXPERT * head["n_active_mean"]
+                                     if (T, H, I, E, K) == (16, 2048, 1024, 64, 8) else None),
+                         "traffic_source": "ncu capture, scaled by active experts",
                          "peak_source": P["source"], "bytes_per_call": head["ffn_bytes_per_call"],
                          "ms_per_call": head["ffn_ms_per_call"]},
             "cpu_baseline": cpu,
