@@ -1,12 +1,14 @@
 // A7 — router-weighted combine of the k expert outputs of each token, with
 // an optional residual: out[t] = bf16_rn(res[t] + sum_j w[t][j] * y[pos(t,j)]),
-// fp32 expert outputs, fp32 accumulation in increasing j (deterministic). One
-// CTA per token; each thread owns 8 consecutive hidden elements.
+// fp32 expert outputs, fp32 accumulation in increasing j (deterministic). A
+// CTA covers CB_THREADS * 8 hidden elements of one token (grid: tokens x hidden
+// slices, so a small decode batch still spreads over many SMs); each thread
+// owns 8 consecutive elements.
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int CB_THREADS = 256;
+constexpr int CB_THREADS = 64;
 
 __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const float *__restrict__ y,
                                                               const float *__restrict__ topk_w,
@@ -23,7 +25,9 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const float *__rest
     ps[threadIdx.x] = pair_pos[int64_t(t) * k + threadIdx.x];
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < H / 8; c += CB_THREADS) {
+  {
+    const int c = blockIdx.y * CB_THREADS + threadIdx.x;
+    if (c >= H / 8) return;
     float acc[8];
     if (residual) {
       const uint4 r = reinterpret_cast<const uint4 *>(residual + int64_t(t) * H)[c];
@@ -33,6 +37,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const float *__rest
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     }
+#pragma unroll 4
     for (int j = 0; j < k; ++j) {
       const int pos = ps[j];
       if (pos < 0) continue;
@@ -62,7 +67,8 @@ extern "C" int moe_combine(const float *y, const float *topk_w, const int32_t *p
   if (!y || !topk_w || !pair_pos || !out) return set_error(MOE_ERR_INVALID_ARG, "moe_combine: NULL pointer");
   if (!aligned(y, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)))
     return set_error(MOE_ERR_INVALID_ARG, "moe_combine: y, residual and out must be 16-byte aligned");
-  cudaError_t e = launch_pdl(combine_kernel, dim3(T), dim3(CB_THREADS), 0, as_stream(stream), y, topk_w, pair_pos,
+  const dim3 grid(unsigned(T), unsigned((H / 8 + CB_THREADS - 1) / CB_THREADS));
+  cudaError_t e = launch_pdl(combine_kernel, grid, dim3(CB_THREADS), 0, as_stream(stream), y, topk_w, pair_pos,
                              residual, k, H, out);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_combine: %s", cudaGetErrorString(e));
   return check_launch("moe_combine");

@@ -69,11 +69,23 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
       wpre[u] = (e_first < e_hi && hc < chunks) ? __ldg(reinterpret_cast<const uint4 *>(wr + int64_t(e_first) * H) + hc)
                                                  : make_uint4(0, 0, 0, 0);
     }
-    for (int c = threadIdx.x; c < RT_TOKENS * chunks; c += RT_THREADS) {
-      const int tt = c / chunks, hc = c % chunks;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (tt < nt) v = __ldg(reinterpret_cast<const uint4 *>(x + int64_t(t0 + tt) * H) + hc);
-      reinterpret_cast<uint4 *>(xs + tt * H)[hc] = v;
+    // the 8 tokens' rows, RT_THREADS 16-byte pieces per pass with all of a
+    // batch's loads issued before any store (one round trip, not one per piece)
+    constexpr int XB = 8;
+    for (int c0 = threadIdx.x; c0 < RT_TOKENS * chunks; c0 += RT_THREADS * XB) {
+      uint4 v[XB];
+#pragma unroll
+      for (int u = 0; u < XB; ++u) {
+        const int c = c0 + u * RT_THREADS;
+        const int tt = c / chunks, hc = c % chunks;
+        v[u] = (c < RT_TOKENS * chunks && tt < nt) ? __ldg(reinterpret_cast<const uint4 *>(x + int64_t(t0 + tt) * H) + hc)
+                                                  : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < XB; ++u) {
+        const int c = c0 + u * RT_THREADS;
+        if (c < RT_TOKENS * chunks) reinterpret_cast<uint4 *>(xs + (c / chunks) * H)[c % chunks] = v[u];
+      }
     }
     __syncthreads();
     for (int e = e_lo + warp; e < e_hi; e += RT_THREADS / 32) {
@@ -150,25 +162,21 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
         if (lane == 0) wout[j] = p;
       }
     } else {
-      uint32_t taken = 0;  // bit m: expert lane + 32m already chosen
-      for (int j = 0; j < k; ++j) {
-        float bk = -INFINITY;
-        int be = 0x7fffffff;
-        for (int m = 0; lane + 32 * m < E; ++m) {
-          const int e = lane + 32 * m;
-          if (!(taken >> m & 1u) && key_better(keys[e], e, bk, be)) { bk = keys[e]; be = e; }
+      // the rank of each key in the order (key descending, expert ascending)
+      // is its place among the top-k: count the keys that beat it
+      for (int e = lane; e < E; e += 32) {
+        const float ke = keys[e];
+        int rank = 0;
+        for (int j = 0; j < E; ++j) rank += key_better(keys[j], j, ke, e) ? 1 : 0;
+        if (rank < k) {
+          const float p = expf(ke - mx) / sum;
+          ids[rank] = e;
+          wout[rank] = p;
+          wsum += p;
         }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-          const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-          if (key_better(ok, oe, bk, be)) { bk = ok; be = oe; }
-        }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        const float p = expf(bk - mx) / sum;
-        wsum += p;
-        if (lane == 0) { ids[j] = be; wout[j] = p; }
       }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     }
     if (flags & MOE_RENORM) {
       __syncwarp();
