@@ -88,8 +88,10 @@ def _route_gpu(M, x, wr, k, bias=None, flags=0, logits_in=None, ids_in=None):
 
 @pytest.mark.parametrize("T,H,E,k,renorm,skew", [
     (37, 2048, 64, 8, False, False), (1, 2048, 64, 8, False, False), (29, 4096, 8, 2, False, False),
-    (29, 4096, 8, 2, True, False), (64, 2048, 64, 8, False, True), (9, 256, 256, 32, True, False)])
+    (29, 4096, 8, 2, True, False), (64, 2048, 64, 8, False, True), (9, 256, 256, 32, True, False),
+    (65, 2048, 64, 8, False, False), (300, 2048, 64, 8, True, True)])
 def test_route_topk(M, T, H, E, k, renorm, skew):
+    # T <= 64 runs 2 tokens per cluster, larger T 8 (both kernels covered)
     x = synth.activations(T, H, seed=3 + T)
     wr = synth.router_weight(0, E, H)
     bias = synth.zipf_log_bias(E) if skew else None

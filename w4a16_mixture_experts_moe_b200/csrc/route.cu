@@ -3,8 +3,10 @@
 // procedure is unchanged; Figure 1 caption: the original BF16 router selects
 // the experts).
 //
-// One thread-block cluster of 8 CTAs serves 8 tokens. CTA rank r computes the
-// logits of experts [r*EPC, (r+1)*EPC) (EPC = ceil(E/8)) for all 8 tokens:
+// One thread-block cluster of 8 CTAs serves TOK tokens (8 for large batches;
+// 2 for decode-sized ones, so their few tokens still spread over many SMs).
+// CTA rank r computes the logits of experts [r*EPC, (r+1)*EPC)
+// (EPC = ceil(E/8)) for all TOK tokens:
 // the tokens' activations are staged in shared memory, each warp takes one
 // expert at a time with every lane's slice of the router row loaded at once
 // (fp32 sums, one BF16 rounding per logit). After a cluster barrier, CTA r
@@ -20,8 +22,7 @@ namespace cg = cooperative_groups;
 
 namespace moe {
 
-constexpr int RT_TOKENS = 8;   // tokens per cluster (one per CTA for top-k)
-constexpr int RT_CLUSTER = 8;  // CTAs per cluster
+constexpr int RT_CLUSTER = 8;  // CTAs per cluster (at most one token per CTA for top-k)
 constexpr int RT_THREADS = 256;
 constexpr int RT_MAX_EPC = MAX_E / RT_CLUSTER;
 
@@ -37,26 +38,27 @@ __device__ __forceinline__ float dot8(const uint4 &w, const uint4 &x, float a) {
   return a;
 }
 
+template <int TOK>
 __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
     route_topk_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, int T, int H, int E, int k,
                       const float *__restrict__ bias, int flags, uint16_t *__restrict__ logits,
                       int32_t *__restrict__ topk_ids, float *__restrict__ topk_w) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ float part[RT_TOKENS][RT_MAX_EPC];  // this CTA's logits (as fp32 of the BF16 value)
+  __shared__ float part[TOK][RT_MAX_EPC];  // this CTA's logits (as fp32 of the BF16 value)
   __shared__ float keys[MAX_E];                   // the token this CTA ranks
   cg::cluster_group cluster = cg::this_cluster();
   pdl_trigger();
   pdl_wait();
   const int rank = int(cluster.block_rank());
-  const int t0 = (blockIdx.x / RT_CLUSTER) * RT_TOKENS;
-  const int nt = min(RT_TOKENS, T - t0);
+  const int t0 = (blockIdx.x / RT_CLUSTER) * TOK;
+  const int nt = min(TOK, T - t0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int EPC = (E + RT_CLUSTER - 1) / RT_CLUSTER;
   const int e_lo = rank * EPC, e_hi = min(E, e_lo + EPC);
   const bool given = flags & MOE_LOGITS_GIVEN;
 
   if (!given) {
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [RT_TOKENS][H]
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [TOK][H]
     const int chunks = H / 8;
     // this warp's first router row: its loads go out before the activations'
     // so the two round trips overlap
@@ -72,26 +74,26 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
     // the 8 tokens' rows, RT_THREADS 16-byte pieces per pass with all of a
     // batch's loads issued before any store (one round trip, not one per piece)
     constexpr int XB = 8;
-    for (int c0 = threadIdx.x; c0 < RT_TOKENS * chunks; c0 += RT_THREADS * XB) {
+    for (int c0 = threadIdx.x; c0 < TOK * chunks; c0 += RT_THREADS * XB) {
       uint4 v[XB];
 #pragma unroll
       for (int u = 0; u < XB; ++u) {
         const int c = c0 + u * RT_THREADS;
         const int tt = c / chunks, hc = c % chunks;
-        v[u] = (c < RT_TOKENS * chunks && tt < nt) ? __ldg(reinterpret_cast<const uint4 *>(x + int64_t(t0 + tt) * H) + hc)
+        v[u] = (c < TOK * chunks && tt < nt) ? __ldg(reinterpret_cast<const uint4 *>(x + int64_t(t0 + tt) * H) + hc)
                                                   : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int u = 0; u < XB; ++u) {
         const int c = c0 + u * RT_THREADS;
-        if (c < RT_TOKENS * chunks) reinterpret_cast<uint4 *>(xs + (c / chunks) * H)[c % chunks] = v[u];
+        if (c < TOK * chunks) reinterpret_cast<uint4 *>(xs + (c / chunks) * H)[c % chunks] = v[u];
       }
     }
     __syncthreads();
     for (int e = e_lo + warp; e < e_hi; e += RT_THREADS / 32) {
-      float acc[RT_TOKENS];
+      float acc[TOK];
 #pragma unroll
-      for (int tt = 0; tt < RT_TOKENS; ++tt) acc[tt] = 0.f;
+      for (int tt = 0; tt < TOK; ++tt) acc[tt] = 0.f;
       const uint4 *wrow = reinterpret_cast<const uint4 *>(wr + int64_t(e) * H);
       int hc = lane;
       for (; hc + 32 * 7 < chunks; hc += 32 * 8) {  // eight 16-byte loads in flight per lane
@@ -102,17 +104,17 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
 #pragma unroll
         for (int u = 0; u < 8; ++u)
 #pragma unroll
-          for (int tt = 0; tt < RT_TOKENS; ++tt)
+          for (int tt = 0; tt < TOK; ++tt)
             acc[tt] = dot8(wv[u], reinterpret_cast<const uint4 *>(xs + tt * H)[hc + 32 * u], acc[tt]);
       }
       for (; hc < chunks; hc += 32) {
         const uint4 wv = __ldg(wrow + hc);
 #pragma unroll
-        for (int tt = 0; tt < RT_TOKENS; ++tt)
+        for (int tt = 0; tt < TOK; ++tt)
           acc[tt] = dot8(wv, reinterpret_cast<const uint4 *>(xs + tt * H)[hc], acc[tt]);
       }
 #pragma unroll
-      for (int tt = 0; tt < RT_TOKENS; ++tt) {
+      for (int tt = 0; tt < TOK; ++tt) {
         float a = acc[tt];
 #pragma unroll
         for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
@@ -204,16 +206,23 @@ extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T
     return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk: NULL pointer");
   if (need_x && (!aligned(x, 16) || !aligned(w_router, 16)))
     return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk: x and w_router must be 16-byte aligned");
-  const size_t smem = need_x ? size_t(RT_TOKENS) * H * 2 : 0;
+  const bool small = T <= 64;  // decode-sized: 2 tokens per cluster
+  const int tok = small ? 2 : 8;
+  const size_t smem = need_x ? size_t(tok) * H * 2 : 0;
   if (smem > 200 * 1024) return set_error(MOE_ERR_SHAPE, "moe_route_topk: H=%d too large", H);
   if (smem > 48 * 1024) {
-    int st = allow_dynamic_smem(reinterpret_cast<const void *>(route_topk_kernel), smem, "moe_route_topk");
+    int st = allow_dynamic_smem(small ? reinterpret_cast<const void *>(route_topk_kernel<2>)
+                                      : reinterpret_cast<const void *>(route_topk_kernel<8>),
+                                smem, "moe_route_topk");
     if (st != MOE_OK) return st;
   }
-  const int64_t blocks = int64_t((T + RT_TOKENS - 1) / RT_TOKENS) * RT_CLUSTER;
+  const int64_t blocks = int64_t((T + tok - 1) / tok) * RT_CLUSTER;
   if (blocks > 0x7fffffffLL) return set_error(MOE_ERR_SHAPE, "moe_route_topk: T too large");
-  const cudaError_t e = launch_pdl(route_topk_kernel, dim3(unsigned(blocks)), dim3(RT_THREADS), smem,
-                                   as_stream(stream), x, w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w);
+  const cudaError_t e =
+      small ? launch_pdl(route_topk_kernel<2>, dim3(unsigned(blocks)), dim3(RT_THREADS), smem, as_stream(stream), x,
+                         w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w)
+            : launch_pdl(route_topk_kernel<8>, dim3(unsigned(blocks)), dim3(RT_THREADS), smem, as_stream(stream), x,
+                         w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_route_topk: %s", cudaGetErrorString(e));
   return check_launch("moe_route_topk");
 }
