@@ -150,17 +150,26 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
       if (i < ngrp) issue(i);
       cp_async_commit();
     }
+    // the lane's activations one group ahead (registers; L2 latency hidden
+    // behind the current group's math)
+    uint4 xn[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      xn[q] = ok && ngrp > 0 ? __ldg(reinterpret_cast<const uint4 *>(xr + kq * GROUP) + q) : make_uint4(0, 0, 0, 0);
     for (int i = 0; i < ngrp; ++i) {
       const int grp = kq + i * KS;
       if (i + GV_DEPTH - 1 < ngrp) issue(i + GV_DEPTH - 1);
       cp_async_commit();
+      uint4 xb[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xb[q] = xn[q];
+      if (ok && i + 1 < ngrp) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xn[q] = __ldg(reinterpret_cast<const uint4 *>(xr + (grp + KS) * GROUP) + q);
+      }
       cp_async_wait<GV_DEPTH - 1>();  // group i's copies (this lane's) have landed
       const uint4 *sr = ring + (i % GV_DEPTH) * (4 * 32) + lane;
       const uint4 g0 = sr[0], g1 = sr[32], u0 = sr[64], u1 = sr[96];
-      uint4 xb[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        xb[q] = ok ? __ldg(reinterpret_cast<const uint4 *>(xr + grp * GROUP) + q) : make_uint4(0, 0, 0, 0);
       float pg[4] = {0.f, 0.f, 0.f, 0.f}, pu[4] = {0.f, 0.f, 0.f, 0.f};
       mma_group(pg, g0, g1, xb);
       mma_group(pu, u0, u1, xb);
