@@ -305,14 +305,18 @@ static cudaError_t launch_gemv_pair(const FfnArgs &a, cudaStream_t s) {
 
 // Warps that share a 16-row slice, from the expected number of active experts
 // E (1 - (1 - k/E)^T): enough warps to keep every SM streaming when a decode
-// step touches few experts.
+// step touches few experts (same-box measurements on the OLMoE decode stack
+// chose the thresholds).
 static int pick_ksplit(const FfnArgs &a) {
   const double miss = 1.0 - double(a.k) / double(a.E);
   double n_act = double(a.E) * (1.0 - std::pow(miss, double(a.T)));
   if (n_act < 1.0) n_act = 1.0;
   const double warps = n_act * (a.I / 16);
   const double want = 148.0 * 24.0;
-  return warps * 2 <= want ? 4 : (warps * 1.25 <= want ? 2 : 1);
+  // with 4+ rows per expert on average (several token chunks per CTA) two
+  // warps per slice shorten each CTA's life enough to pay for the reduction
+  const bool many_rows = int64_t(a.T) * a.k >= 4 * int64_t(a.E);
+  return warps * 2 <= want ? 4 : (warps * 1.25 <= want || many_rows ? 2 : 1);
 }
 
 int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s) {
