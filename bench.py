@@ -67,6 +67,7 @@ def parse():
                          "slotcache: 16 layers decoding from a pinned host pool through S GPU slots per layer")
     ap.add_argument("--slots", type=int, default=16)
     ap.add_argument("--shape", default="olmoe", choices=list(SHAPES))
+    ap.add_argument("--skew", action="store_true", help="prefill with Zipf(1.2) log-bias routing")
     a = ap.parse_args()
     if a.workload == "prefill" and a.T == 16:
         a.T = 8192
@@ -181,7 +182,7 @@ class Stack:
     """16 OLMoE-shaped layers: per layer a packed expert bank and a router, plus
     per-T buffers. Weights are drawn on the device with the seeded recipe."""
 
-    def __init__(self, layers, path, shape="olmoe", renorm=False):
+    def __init__(self, layers, path, shape="olmoe", renorm=False, skew=False):
         import torch
 
         import synth
@@ -191,6 +192,8 @@ class Stack:
         H, I, E, K = SHAPES[shape]
         self.H, self.I, self.E, self.K = H, I, E, K
         self.flags = M.MOE_RENORM if renorm else 0
+        # skewed routing: log Zipf(1.2) per-expert offsets added to the logits
+        self.bias = torch.from_numpy(synth.zipf_log_bias(E)).float().cuda() if skew else None
         self.path = {"auto": M.MOE_PATH_AUTO, "gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC}[path]
         self.banks, self.routers = [], []
         for l in range(layers):
@@ -216,7 +219,8 @@ class Stack:
         cur = x_in
         for l in range(self.layers):
             out = xs[l % 2] if cur is not xs[l % 2] else xs[(l + 1) % 2]
-            moe_layer_forward(cur, self.routers[l], self.banks[l], bufs[l], flags=self.flags, residual=cur, out=out)
+            moe_layer_forward(cur, self.routers[l], self.banks[l], bufs[l], bias=self.bias, flags=self.flags,
+                              residual=cur, out=out)
             cur = out
         return cur
 
@@ -291,6 +295,7 @@ def measure_T(stack, T, steps, warmup, world, want_e2e=True, want_roofline=True)
         n_act = [int((b.counts > 0).sum().item()) for b in bufs]
         res["ffn_ms_per_call"] = ms_ffn_layers / stack.layers
         res["n_active_mean"] = statistics.mean(n_act)
+        res["counts_layer0"] = [int(c) for c in bufs[0].counts.tolist()]
         res["ffn_bytes_per_call"] = statistics.mean(n_act) * rec_bytes(stack.H, stack.I)
         res["ffn_flops_per_call"] = 6.0 * T * stack.K * stack.H * stack.I
     del g, g2
@@ -520,7 +525,7 @@ def main_slotcache(a, rank, world, P):
 def main_prefill(a, rank, world, P):
     """One layer at large T (tensor-core path); roofline = FLOPs / FFN time."""
     H_, I_, E_, K_ = SHAPES[a.shape]
-    stack = Stack(a.layers, a.path, a.shape, renorm=(a.shape == "wide"))
+    stack = Stack(a.layers, a.path, a.shape, renorm=(a.shape == "wide"), skew=a.skew)
     r = measure_T(stack, a.T, a.steps, a.warmup, world)
     if rank == 0:
         T, L = a.T, a.layers
@@ -529,7 +534,8 @@ def main_prefill(a, rank, world, P):
             "metric": METRIC, "value": T * L * world / (r["ms_per_step"] / 1e3), "unit": "layer-tokens/s",
             "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{a.shape}-prefill", "T": T, "layers": L, "H": H_, "I": I_, "E": E_, "k": K_,
+            "config": {"workload": f"{a.shape}-prefill" + ("-zipf1.2-skew" if a.skew else ""), "T": T, "layers": L,
+                       "H": H_, "I": I_, "E": E_, "k": K_,
                        "weights": "int4 group-128 symmetric, all experts resident",
                        "l2": f"inputs larger than L2 ({E_ * rec_bytes(H_, I_) / 1e6:.0f} MB of packed experts)",
                        "parallelism": f"replicas{world}"},
@@ -545,6 +551,10 @@ def main_prefill(a, rank, world, P):
             "gpu_launches": r["launches_per_step"] * a.steps,
             "clocks": r["clocks"],
         }
+        if a.skew:
+            c = r["counts_layer0"]
+            line["routing"] = {"bias": "log Zipf(s=1.2) per expert", "n_active": sum(1 for v in c if v > 0),
+                               "max_group": max(c), "empty_groups": sum(1 for v in c if v == 0), "histogram": c}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
