@@ -45,10 +45,11 @@
 // MOE_DEVERR_RANGE for an activation out of range. The gate/up epilogue
 // rounds h to BF16 (the method's A16 intermediate) and stores that value in
 // FP16, which again is exact.
-// The down pass keeps two accumulator buffers so the epilogue of tile i
-// overlaps the mainloop of tile i+1; gate + up at N = 256 fill all 512
-// tensor-memory columns with one buffer, so there the epilogue is kept short
-// (eight warps, fast-divide SiLU) instead. Every wait is bounded (about two
+// Both passes run two 128-row blocks of A against each activation box (gate
+// and up of the same features; or 256 consecutive down-output features), so
+// the two N = 256 accumulators fill all 512 tensor-memory columns with one
+// buffer: the epilogue is kept short (eight warps, fast-divide SiLU) instead
+// of overlapped. Every wait is bounded (about two
 // seconds of %globaltimer); a wait that runs out flags MOE_DEVERR_TIMEOUT and
 // all roles drain and exit.
 #include <cuda.h>
@@ -78,19 +79,24 @@ constexpr uint64_t WAIT_NS = 2000000000ull;
 
 template <bool GATEUP>
 struct Cfg {
-  static constexpr int NMAT = GATEUP ? 2 : 1;
+  // A holds two 128-row blocks: gate and up rows of the same 128 features
+  // (gate/up pass), or two consecutive 128-row blocks of the down matrix (down
+  // pass: 256 output features per tile, so each activation box feeds twice
+  // the MMA work)
+  static constexpr int NMAT = 2;
   static constexpr int A_BYTES = NMAT * BM * BK * 2;  // 16 KB per matrix
   static constexpr int B_BYTES = BN * BK * 2;         // 32 KB
   static constexpr int C_BYTES = NMAT * BM * BK / 2;  // 4 KB of codes per matrix
-  static constexpr int S = GATEUP ? 3 : 4;            // A and B ring depth (one commit frees both)
-  static constexpr int CS = GATEUP ? 3 : 4;           // codes ring depth
+  static constexpr int S = 3;                         // A and B ring depth (one commit frees both)
+  static constexpr int CS = 3;                        // codes ring depth
+  static constexpr int FW = GATEUP ? BM : 2 * BM;     // output features per tile
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = A_OFF + S * A_BYTES;
   static constexpr int C_OFF = B_OFF + S * B_BYTES;
   static constexpr int RING_BYTES = C_OFF + CS * C_BYTES;
   static constexpr int ACC_COLS = NMAT * BN;          // columns per accumulator buffer
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NBUF = TMEM_COLS / ACC_COLS;   // 1 (gate/up) or 2 (down) accumulator buffers
+  static constexpr int NBUF = TMEM_COLS / ACC_COLS;   // accumulator buffers (1: two N = 256 blocks fill TMEM)
   static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 4096 /*tables, barriers*/;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(S <= MAX_RING && CS <= MAX_RING, "ring depth");
@@ -242,6 +248,7 @@ struct Tile {
   int e, lo, n0, nvalid, f0;
 };
 
+template <int FW>
 __device__ __forceinline__ Tile decode_tile(const Shared &sh, int E, int FT, int t) {
   int lo_e = 0, hi_e = E;  // largest e with tstart[e] <= t
   while (hi_e - lo_e > 1) {
@@ -253,15 +260,16 @@ __device__ __forceinline__ Tile decode_tile(const Shared &sh, int E, int FT, int
   const int r = t - sh.tstart[lo_e];
   x.lo = sh.off[lo_e];
   x.n0 = (r / FT) * BN;
-  x.f0 = (r % FT) * BM;
+  x.f0 = (r % FT) * FW;
   x.nvalid = min(BN, sh.off[lo_e + 1] - x.lo - x.n0);
   return x;
 }
 
 // tm_b: activation rows in group order (gate/up: FP16 x gathered by the
 // pre-pass; down: h), box 64 x 256, 128-byte swizzle. tm_q0 / tm_q1: packed
-// codes of the first / second matrix over the record bank, box 32 B x 128
-// rows x 1 record.
+// codes of A's first / second 128-row block over the record bank (gate and up;
+// or the down matrix twice, at rows f0 and f0 + 128), box 32 B x 128 rows x 1
+// record.
 template <bool GATEUP>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_ffn_kernel(const FfnArgs a, const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_q0,
@@ -274,7 +282,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int E = a.E;
   const int NOUT = GATEUP ? a.I : a.H;   // output features
   const int KD = GATEUP ? a.H : a.I;     // reduction length
-  const int FT = NOUT / BM;              // feature tiles per token tile
+  const int FT = (NOUT + C::FW - 1) / C::FW;  // feature tiles per token tile
   const int KS = KD / BK;                // k-steps per tile
   const int G = KD / GROUP;
   pdl_trigger();
@@ -355,13 +363,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ks == KS || deq_tile < 0) {
         ks = 0;
         ++deq_tile;
-        const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + deq_tile * int(gridDim.x));
+        const Tile tl = decode_tile<C::FW>(sh, E, FT, int(blockIdx.x) + deq_tile * int(gridDim.x));
         const int slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
         const uint8_t *rec = a.bank + int64_t(slot) * a.rec;
-        deq_srow = reinterpret_cast<const uint16_t *>(rec + (GATEUP ? (p ? a.off_us : a.off_gs) : a.off_ds)) +
-                   int64_t(tl.f0 + i) * G;
+        // row of this thread's weights; down rows past H (a ragged last
+        // tile) get a zero scale, their codes arrive as zeros
+        const int row = tl.f0 + (GATEUP ? 0 : p * BM) + i;
+        deq_srow = row < NOUT ? reinterpret_cast<const uint16_t *>(rec + (GATEUP ? (p ? a.off_us : a.off_gs) : a.off_ds)) +
+                                    int64_t(row) * G
+                              : nullptr;
       }
-      const uint16_t sbits = deq_srow[(ks * BK) / GROUP];  // one 32-byte line per row and tile
+      const uint16_t sbits = deq_srow ? deq_srow[(ks * BK) / GROUP] : uint16_t(0);  // one 32-byte line per row and tile
       const int cs = it % C::CS, as = it % C::S;
       // wait results are made warp-uniform: a lane never leaves the loop
       // while the rest of its warp goes on to a __syncwarp
@@ -369,25 +381,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       const uint8_t *nib = ringC + cs * C::C_BYTES;  // [matrix][128 rows][32 B]
       uint32_t words[8];
-      if (GATEUP) {
+      {
         const uint8_t *src = nib + (p * BM + i) * 32;
         const uint4 w0 = *reinterpret_cast<const uint4 *>(src);
         const uint4 w1 = *reinterpret_cast<const uint4 *>(src + 16);
         words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
         words[4] = w1.x; words[5] = w1.y; words[6] = w1.z; words[7] = w1.w;
-      } else {
-        const uint4 w0 = *reinterpret_cast<const uint4 *>(nib + i * 32 + p * 16);
-        words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
-        words[4] = words[5] = words[6] = words[7] = 0;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.c_free[cs]);  // the warp's codes are in registers: the slot may be refilled
       ok = __all_sync(0xffffffffu, wait_bounded(sh, &sh.s_free[as], ((it / C::S) & 1) ^ 1, a.err));
       if (!ok) break;
       const __half2 sc = __half2half2(__float2half_rn(bf16_to_f(sbits)));
-      constexpr int NW = GATEUP ? 8 : 4;
-      const int c0 = GATEUP ? 0 : 4 * p;
-      uint8_t *arow = ringA + as * C::A_BYTES + (GATEUP ? p * (BM * BK * 2) : 0) + i * 128;
+      constexpr int NW = 8;
+      const int c0 = 0;
+      uint8_t *arow = ringA + as * C::A_BYTES + p * (BM * BK * 2) + i * 128;
 #pragma unroll
       for (int wd = 0; wd < NW; ++wd) {
         // k = 2i + h sits at bits 4(i + 4h): OR-ing the nibbles at bits 0-3 /
@@ -419,7 +427,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int frow = q * 32 + lane;                  // feature within the tile
     for (int tl_i = 0; tl_i < my_tiles; ++tl_i) {
       const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
-      const Tile tl = decode_tile(sh, E, FT, t);
+      const Tile tl = decode_tile<C::FW>(sh, E, FT, t);
       const int b = tl_i % C::NBUF;
       if (!__all_sync(0xffffffffu, wait_bounded(sh, &sh.tmem_full[b], (tl_i / C::NBUF) & 1, a.err))) break;
       tc_fence_after();
@@ -444,11 +452,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         } else {
+          uint32_t g2[16];
+          tmem_ld16(tbase + BN + j0, g2);  // second 128-row block
           tmem_wait_ld();
           float *yp = a.y + (row0 + j0) * NOUT + f;
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj)
             if (j0 + jj < j_hi) yp[jj * NOUT] = __uint_as_float(g[jj]);
+          if (f + BM < NOUT) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              if (j0 + jj < j_hi) yp[jj * NOUT + BM] = __uint_as_float(g2[jj]);
+          }
         }
       }
       tc_fence_before();
@@ -500,7 +515,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int it = 0; it < iters; ++it) {
       bool ok = true;
       if (ks == 0) {
-        const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + tl_i * int(gridDim.x));
+        const Tile tl = decode_tile<C::FW>(sh, E, FT, int(blockIdx.x) + tl_i * int(gridDim.x));
         n16 = max(1, (tl.nvalid + 15) >> 4);
         ok = wait_bounded(sh, &sh.tmem_empty[tl_i % C::NBUF], ((tl_i / C::NBUF) & 1) ^ 1, a.err);
       }
@@ -528,7 +543,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (cur < 0 || ks == KS) {
         ks = 0;
         ++cur;
-        const Tile tl = decode_tile(sh, E, FT, int(blockIdx.x) + cur * int(gridDim.x));
+        const Tile tl = decode_tile<C::FW>(sh, E, FT, int(blockIdx.x) + cur * int(gridDim.x));
         slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
         row_b = tl.lo + tl.n0;  // first activation row of the tile, in group order
         f0 = tl.f0;
@@ -538,7 +553,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint8_t *dst = ringC + s * C::C_BYTES;
           mbar_arrive_expect_tx(&loaded[s], C::C_BYTES);
           tma_load_3d(dst, &tm_q0, ks * (BK / 2), f0, slot, &loaded[s]);
-          if (GATEUP) tma_load_3d(dst + BM * (BK / 2), &tm_q1, ks * (BK / 2), f0, slot, &loaded[s]);
+          tma_load_3d(dst + BM * (BK / 2), &tm_q1, ks * (BK / 2), f0 + (GATEUP ? 0 : BM), slot, &loaded[s]);
         } else {
           mbar_arrive_expect_tx(&loaded[s], C::B_BYTES);
           tma_load_2d(ringB + s * C::B_BYTES, &tm_b, ks * BK, row_b, &loaded[s]);
