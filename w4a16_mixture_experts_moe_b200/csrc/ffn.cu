@@ -39,22 +39,33 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *__restric
 
 // xs[r] = FP16(x[sorted_pair[r] / k]) for the P rows in group order: the
 // tensor-core gate/up pass then loads each token tile of an expert as one
-// contiguous block of rows.
+// contiguous block of rows. One warp per row (grid-stride over rows); each
+// lane issues all its loads of a pass before converting and storing, so a
+// row costs one round trip rather than one per 16-byte piece.
 __global__ void __launch_bounds__(256) gather_x_f16_kernel(const uint16_t *__restrict__ x,
                                                            const int32_t *__restrict__ sorted_pair, int k, int T,
-                                                           int H8, int64_t n8, uint16_t *__restrict__ xs,
+                                                           int H8, int64_t P, uint16_t *__restrict__ xs,
                                                            int32_t *err) {
   pdl_trigger();
   pdl_wait();
+  constexpr int U = 8;
   bool bad = false;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = i / H8;
-    const int c = int(i - r * H8);
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5; r < P; r += nw) {
     const int t = sorted_pair[r] / k;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (t >= 0 && t < T) v = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4 *>(x + int64_t(t) * H8 * 8) + c), bad);
-    else flag_error(err, MOE_DEVERR_EXPERT_ID);
-    reinterpret_cast<uint4 *>(xs)[i] = v;
+    const bool ok = t >= 0 && t < T;
+    if (!ok && lane == 0) flag_error(err, MOE_DEVERR_EXPERT_ID);
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + int64_t(ok ? t : 0) * H8 * 8);
+    uint4 *dst = reinterpret_cast<uint4 *>(xs) + r * H8;
+    for (int c0 = lane; c0 < H8; c0 += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = c0 + 32 * u < H8 ? __ldg(src + c0 + 32 * u) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + 32 * u < H8) dst[c0 + 32 * u] = ok ? bf16x8_to_f16x8(v[u], bad) : make_uint4(0, 0, 0, 0);
+    }
   }
   if (bad) flag_error(err, MOE_DEVERR_RANGE);
 }
@@ -78,11 +89,11 @@ int launch_x_to_f16(const FfnArgs &a, cudaStream_t s) {
 }
 
 int launch_gather_x_f16(const FfnArgs &a, cudaStream_t s) {
-  const int64_t n8 = int64_t(a.T) * a.k * a.H / 8;
-  const int64_t want = (n8 + 255) / 256, cap = 148 * 8;
+  const int64_t P = int64_t(a.T) * a.k;
+  const int64_t want = (P + 7) / 8, cap = 148 * 16;  // 8 rows (warps) per block
   const int blocks = int(want < cap ? (want > 0 ? want : 1) : cap);
   const cudaError_t e =
-      launch_pdl(gather_x_f16_kernel, dim3(blocks), dim3(256), 0, s, a.x, a.sorted_pair, a.k, a.T, a.H / 8, n8, a.xs, a.err);
+      launch_pdl(gather_x_f16_kernel, dim3(blocks), dim3(256), 0, s, a.x, a.sorted_pair, a.k, a.T, a.H / 8, P, a.xs, a.err);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (gather x): %s", cudaGetErrorString(e));
   return check_launch("moe_grouped_w4a16_ffn (gather x)");
 }

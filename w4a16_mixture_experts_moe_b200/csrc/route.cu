@@ -38,6 +38,49 @@ __device__ __forceinline__ float dot8(const uint4 &w, const uint4 &x, float a) {
   return a;
 }
 
+// Softmax over all E keys and the top-k of one token, by one warp. keys: the
+// token's fp32 logits (+ bias, NaN turned into -inf) in shared memory. The
+// rank of each key in the order (key descending, expert ascending) is its
+// place among the top-k: each lane counts the keys that beat each of its own.
+// With MOE_IDS_GIVEN the ids are read and only their weights are written.
+__device__ void topk_warp(const float *keys, int E, int k, int flags, int32_t *ids, float *wout, int lane) {
+  float mx = -INFINITY;
+  for (int e = lane; e < E; e += 32) mx = fmaxf(mx, keys[e]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+  for (int e = lane; e < E; e += 32) sum += expf(keys[e] - mx);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  float wsum = 0.f;
+  if (flags & MOE_IDS_GIVEN) {
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[j];
+      const float p = (e >= 0 && e < E) ? expf(keys[e] - mx) / sum : 0.f;
+      wsum += p;
+      if (lane == 0) wout[j] = p;
+    }
+  } else {
+    for (int e = lane; e < E; e += 32) {
+      const float ke = keys[e];
+      int rank = 0;
+      for (int j = 0; j < E; ++j) rank += key_better(keys[j], j, ke, e) ? 1 : 0;
+      if (rank < k) {
+        const float p = expf(ke - mx) / sum;
+        ids[rank] = e;
+        wout[rank] = p;
+        wsum += p;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+  }
+  if (flags & MOE_RENORM) {
+    __syncwarp();
+    for (int j = lane; j < k; j += 32) wout[j] = wout[j] / wsum;
+  }
+}
+
 template <int TOK>
 __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
     route_topk_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, int T, int H, int E, int k,
@@ -144,48 +187,122 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
       keys[e] = v;
     }
     __syncwarp();
-    float mx = -INFINITY;
-    for (int e = lane; e < E; e += 32) mx = fmaxf(mx, keys[e]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.f;
-    for (int e = lane; e < E; e += 32) sum += expf(keys[e] - mx);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-
-    int32_t *ids = topk_ids + int64_t(t) * k;
-    float *wout = topk_w + int64_t(t) * k;
-    float wsum = 0.f;
-    if (flags & MOE_IDS_GIVEN) {
-      for (int j = 0; j < k; ++j) {
-        const int e = ids[j];
-        const float p = (e >= 0 && e < E) ? expf(keys[e] - mx) / sum : 0.f;
-        wsum += p;
-        if (lane == 0) wout[j] = p;
-      }
-    } else {
-      // the rank of each key in the order (key descending, expert ascending)
-      // is its place among the top-k: count the keys that beat it
-      for (int e = lane; e < E; e += 32) {
-        const float ke = keys[e];
-        int rank = 0;
-        for (int j = 0; j < E; ++j) rank += key_better(keys[j], j, ke, e) ? 1 : 0;
-        if (rank < k) {
-          const float p = expf(ke - mx) / sum;
-          ids[rank] = e;
-          wout[rank] = p;
-          wsum += p;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-    }
-    if (flags & MOE_RENORM) {
-      __syncwarp();
-      for (int j = lane; j < k; j += 32) wout[j] = wout[j] / wsum;
-    }
+    topk_warp(keys, E, k, flags, topk_ids + int64_t(t) * k, topk_w + int64_t(t) * k, lane);
   }
   cluster.sync();  // keep this CTA's shared memory alive until every reader is done
+}
+
+// ---------------------------------------------------------------- large batches
+// For T > 64 the logits are a real GEMM (T x H by H x E): warp-level tensor-core
+// MMAs (mma.sync m16n8k16, BF16 in, fp32 accumulate, one BF16 rounding per
+// logit, the same arithmetic reading as the cluster kernel), then one warp
+// per token for softmax + top-k.
+constexpr int LG_TM = 64;   // tokens per CTA
+constexpr int LG_TE = 64;   // experts per CTA
+constexpr int LG_KC = 64;   // K per shared-memory chunk
+constexpr int LG_LD = 72;   // padded row (bf16): 144-byte rows, ldmatrix without bank conflicts
+
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// logits[t][e] = bf16_rn(sum_h x[t][h] Wr[e][h]) for a 64 x 64 (token x expert)
+// tile; warp w owns tokens 16w..16w+15 and all 64 experts (8 n-tiles). The K
+// chunks are double-buffered with cp.async; rows past T / E and columns past H
+// read as zero.
+__global__ void __launch_bounds__(128) logits_mma_kernel(const uint16_t *__restrict__ x,
+                                                         const uint16_t *__restrict__ wr, int T, int H, int E,
+                                                         uint16_t *__restrict__ logits) {
+  __shared__ __align__(16) uint16_t xs[2][LG_TM][LG_LD];
+  __shared__ __align__(16) uint16_t ws[2][LG_TE][LG_LD];
+  pdl_trigger();
+  pdl_wait();
+  const int t0 = blockIdx.x * LG_TM, e0 = blockIdx.y * LG_TE;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int nchunk = (H + LG_KC - 1) / LG_KC;
+  auto load = [&](int c, int buf) {  // 64 rows x 64 k of x and of Wr, 16 bytes per copy
+    const int k0 = c * LG_KC;
+    for (int i = threadIdx.x; i < LG_TM * (LG_KC / 8); i += 128) {
+      const int r = i >> 3, cc = i & 7, kk = k0 + cc * 8;
+      const bool vx = t0 + r < T && kk < H, vw = e0 + r < E && kk < H;
+      cp_async16_zfill(&xs[buf][r][cc * 8], x + (vx ? int64_t(t0 + r) * H + kk : 0), vx);
+      cp_async16_zfill(&ws[buf][r][cc * 8], wr + (vw ? int64_t(e0 + r) * H + kk : 0), vw);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  float acc[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
+  load(0, 0);
+  for (int c = 0; c < nchunk; ++c) {
+    const int buf = c & 1;
+    if (c + 1 < nchunk) {
+      load(c + 1, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < LG_KC / 16; ++kk) {
+      uint32_t af[4];
+      ldmatrix_x4(af, &xs[buf][warp * 16 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+#pragma unroll
+      for (int jp = 0; jp < 4; ++jp) {  // two n-tiles of experts per ldmatrix
+        uint32_t bf[4];
+        ldmatrix_x4(bf, &ws[buf][jp * 16 + (lane & 7) + ((lane >> 4) << 3)][kk * 16 + ((lane >> 3) & 1) * 8]);
+        mma_bf16_16816(acc[2 * jp], af, bf[0], bf[1]);
+        mma_bf16_16816(acc[2 * jp + 1], af, bf[2], bf[3]);
+      }
+    }
+    __syncthreads();  // the buffer is refilled next iteration
+  }
+  // accumulator (c0, c1) = token g, experts 2t, 2t+1 of the n-tile; (c2, c3) = token g+8
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int tok = t0 + warp * 16 + g + (c >> 1) * 8;
+      const int e = e0 + j * 8 + 2 * t + (c & 1);
+      if (tok < T && e < E) logits[int64_t(tok) * E + e] = f_to_bf16(acc[j][c]);
+    }
+}
+
+// Softmax + top-k from given logits, one warp per token.
+__global__ void __launch_bounds__(256) topk_kernel(const uint16_t *__restrict__ logits, int T, int E, int k,
+                                                   const float *__restrict__ bias, int flags, int32_t *topk_ids,
+                                                   float *topk_w) {
+  __shared__ float keys[8][MAX_E];
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  for (int e = lane; e < E; e += 32) {
+    float v = bf16_to_f(logits[int64_t(t) * E + e]);
+    if (bias) v = v + bias[e];
+    if (v != v) v = -INFINITY;  // NaN never wins
+    keys[warp][e] = v;
+  }
+  __syncwarp();
+  topk_warp(keys[warp], E, k, flags, topk_ids + int64_t(t) * k, topk_w + int64_t(t) * k, lane);
 }
 
 }  // namespace moe
@@ -206,6 +323,21 @@ extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T
     return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk: NULL pointer");
   if (need_x && (!aligned(x, 16) || !aligned(w_router, 16)))
     return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk: x and w_router must be 16-byte aligned");
+  cudaError_t e;
+  if (T > 64 && (!need_x || H % 16 == 0)) {
+    // large batch: tensor-core logits GEMM (unless given), then top-k per token
+    if (need_x) {
+      e = launch_pdl(logits_mma_kernel, dim3(unsigned((T + LG_TM - 1) / LG_TM), unsigned((E + LG_TE - 1) / LG_TE)),
+                     dim3(128), 0, as_stream(stream), x, w_router, T, H, E, logits);
+      if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_route_topk (logits): %s", cudaGetErrorString(e));
+      const int st = check_launch("moe_route_topk (logits)");
+      if (st != MOE_OK) return st;
+    }
+    e = launch_pdl(topk_kernel, dim3(unsigned((T + 7) / 8)), dim3(256), 0, as_stream(stream), logits, T, E, k, bias,
+                   flags, topk_ids, topk_w);
+    if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_route_topk: %s", cudaGetErrorString(e));
+    return check_launch("moe_route_topk");
+  }
   const bool small = T <= 64;  // decode-sized: 2 tokens per cluster
   const int tok = small ? 2 : 8;
   const size_t smem = need_x ? size_t(tok) * H * 2 : 0;
@@ -218,8 +350,7 @@ extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T
   }
   const int64_t blocks = int64_t((T + tok - 1) / tok) * RT_CLUSTER;
   if (blocks > 0x7fffffffLL) return set_error(MOE_ERR_SHAPE, "moe_route_topk: T too large");
-  const cudaError_t e =
-      small ? launch_pdl(route_topk_kernel<2>, dim3(unsigned(blocks)), dim3(RT_THREADS), smem, as_stream(stream), x,
+  e = small ? launch_pdl(route_topk_kernel<2>, dim3(unsigned(blocks)), dim3(RT_THREADS), smem, as_stream(stream), x,
                          w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w)
             : launch_pdl(route_topk_kernel<8>, dim3(unsigned(blocks)), dim3(RT_THREADS), smem, as_stream(stream), x,
                          w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w);
