@@ -110,13 +110,22 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The largest of the ranks' values (device times: the job's time is the
+    slowest rank's). The reduction runs on the GPU under NCCL, on the host
+    under gloo."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([float(v)], device="cuda")
+    t = torch.tensor([float(v)], device="cuda" if dist.get_backend() == "nccl" else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_value(units_per_rank, world, ms_max):
+    """Whole-job throughput of `world` replicas: all ranks' units over the
+    slowest rank's time (weak scaling: every rank runs the full workload)."""
+    return units_per_rank * world / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -387,7 +396,7 @@ def main():
         dist.barrier()
     if rank == 0:
         T, L = a.T, a.layers
-        value = T * L * world / (head["ms_per_step"] / 1e3)
+        value = replica_value(T * L, world, head["ms_per_step"])
         achieved = head["ffn_bytes_per_call"] / (head["ffn_ms_per_call"] / 1e3) / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": "layer-tokens/s", "n_gpus": world, "steps": a.steps,
@@ -397,7 +406,7 @@ def main():
                        "weights": "int4 group-128 symmetric, all experts resident",
                        "l2": "inputs larger than L2 (3.32 GB of packed experts read per step)",
                        "parallelism": f"replicas{world}"},
-            "e2e": {"value": T * L * world / (head["ms_e2e"] / 1e3), "unit": "layer-tokens/s",
+            "e2e": {"value": replica_value(T * L, world, head["ms_e2e"]), "unit": "layer-tokens/s",
                     "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
             "roofline": {"bound": "hbm", "kernel": "moe_grouped_w4a16_ffn (gate/up + down kernels), per layer call",
                          "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
@@ -531,7 +540,7 @@ def main_prefill(a, rank, world, P):
         T, L = a.T, a.layers
         achieved = r["ffn_flops_per_call"] / (r["ffn_ms_per_call"] / 1e3) / 1e12
         line = {
-            "metric": METRIC, "value": T * L * world / (r["ms_per_step"] / 1e3), "unit": "layer-tokens/s",
+            "metric": METRIC, "value": replica_value(T * L, world, r["ms_per_step"]), "unit": "layer-tokens/s",
             "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{a.shape}-prefill" + ("-zipf1.2-skew" if a.skew else ""), "T": T, "layers": L,
@@ -539,7 +548,7 @@ def main_prefill(a, rank, world, P):
                        "weights": "int4 group-128 symmetric, all experts resident",
                        "l2": f"inputs larger than L2 ({E_ * rec_bytes(H_, I_) / 1e6:.0f} MB of packed experts)",
                        "parallelism": f"replicas{world}"},
-            "e2e": {"value": T * L * world / (r["ms_e2e"] / 1e3), "unit": "layer-tokens/s",
+            "e2e": {"value": replica_value(T * L, world, r["ms_e2e"]), "unit": "layer-tokens/s",
                     "h2d_bytes_per_step": T * H_ * 2, "d2h_bytes_per_step": T * H_ * 2},
             "roofline": {"bound": "tensor", "kernel": "moe_grouped_w4a16_ffn (tcgen05 gate/up + down), per call",
                          "achieved": achieved, "peak": P["bf16_tflops"], "unit": "TFLOP/s",
