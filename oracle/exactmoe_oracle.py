@@ -327,14 +327,19 @@ def grouped_ffn(x, experts: PackedExperts, sorted_pair, offsets, k: int):
 
 
 def combine(y_sorted, w, pair_pos, residual=None) -> np.ndarray:
-    """out[t] = bf16_rn(residual[t] + sum_j w[t][j] * y[pair_pos[t*k+j]]), j in order."""
+    """out[t] = bf16_rn(residual[t] + sum_j w[t][j] * y[pair_pos[t*k+j]]), j in order.
+
+    A pair with pair_pos < 0 (dropped by the grouping because its expert id
+    was out of range, which the library flags) contributes nothing.
+    """
     w = np.asarray(w, dtype=np.float64)
     T, k = w.shape
     y = np.asarray(y_sorted, dtype=np.float64)
     pos = np.asarray(pair_pos, dtype=np.int64).reshape(T, k)
     acc = np.zeros((T, y.shape[1])) if residual is None else np.array(residual, dtype=np.float64)
     for j in range(k):
-        acc = acc + w[:, j:j + 1] * y[pos[:, j]]
+        keep = (pos[:, j] >= 0)[:, None]
+        acc = acc + np.where(keep, w[:, j:j + 1] * y[np.maximum(pos[:, j], 0)], 0.0)
     return round_to_bf16(acc)
 
 

@@ -248,12 +248,16 @@ def test_grouped_ffn_not_resident_is_flagged(M):
 
 # ------------------------------------------------------------------ A7 combine
 
-@pytest.mark.parametrize("T,k,H,res", [(16, 8, 2048, True), (5, 2, 4096, False), (1, 8, 2048, True)])
-def test_combine(M, T, k, H, res):
+@pytest.mark.parametrize("T,k,H,res,drop", [(16, 8, 2048, True, False), (5, 2, 4096, False, False),
+                                            (1, 8, 2048, True, False), (7, 4, 2048, True, True)])
+def test_combine(M, T, k, H, res, drop):
     rng = np.random.default_rng(T + k)
     y = synth.normal_bf16((T * k, H), 0.5, 77).float() * 1.001   # fp32 values with low bits set
     w = torch.from_numpy(rng.random((T, k)).astype(np.float32))
-    pp = torch.from_numpy(rng.permutation(T * k).astype(np.int32))
+    perm = rng.permutation(T * k).astype(np.int32)
+    if drop:                                                       # dropped pairs contribute nothing
+        perm[[0, 5, 13]] = -1
+    pp = torch.from_numpy(perm)
     r = synth.activations(T, H, seed=78) if res else None
     out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
     M.moe_combine(y.cuda(), w.cuda(), pp.cuda(), None if r is None else r.cuda(), T, k, H, out)

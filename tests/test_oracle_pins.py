@@ -258,3 +258,20 @@ def test_combine_closed_form():
     out = o.combine(y, w, pair_pos, res)
     for t in range(T):
         assert np.all(out[t] == 1 + 0.25 * (2 * t + 1) + 0.5 * (2 * t + 2))
+
+
+def test_combine_dropped_pair_equals_zero_weight():
+    # a pair with pair_pos = -1 contributes exactly what a weight of 0 would
+    rng = np.random.default_rng(5)
+    T, k, H = 4, 3, 8
+    y = rng.standard_normal((T * k, H))
+    w = rng.random((T, k))
+    pos = rng.permutation(T * k).astype(np.int64)
+    res = rng.standard_normal((T, H))
+    dropped = pos.copy()
+    dropped[[1, 7]] = -1                     # pairs (0, 1) and (2, 1)
+    w0 = w.copy()
+    w0[0, 1] = 0.0
+    w0[2, 1] = 0.0
+    assert np.array_equal(o.combine(y, w, dropped, res), o.combine(y, w0, pos, res))
+
