@@ -156,6 +156,9 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       xn[q] = ok && ngrp > 0 ? __ldg(reinterpret_cast<const uint4 *>(xr + kq * GROUP) + q) : make_uint4(0, 0, 0, 0);
+    // the group's four scales, also one group ahead
+    uint16_t sgn0 = 0, sgn1 = 0, sun0 = 0, sun1 = 0;
+    if (ngrp > 0) { sgn0 = gs[kq]; sgn1 = gs[8 * G + kq]; sun0 = us[kq]; sun1 = us[8 * G + kq]; }
     for (int i = 0; i < ngrp; ++i) {
       const int grp = kq + i * KS;
       if (i + GV_DEPTH - 1 < ngrp) issue(i + GV_DEPTH - 1);
@@ -163,9 +166,13 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
       uint4 xb[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) xb[q] = xn[q];
-      if (ok && i + 1 < ngrp) {
+      const float sg0 = bf16_to_f(sgn0), sg1 = bf16_to_f(sgn1), su0 = bf16_to_f(sun0), su1 = bf16_to_f(sun1);
+      if (i + 1 < ngrp) {
+        sgn0 = gs[grp + KS]; sgn1 = gs[8 * G + grp + KS]; sun0 = us[grp + KS]; sun1 = us[8 * G + grp + KS];
+        if (ok) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) xn[q] = __ldg(reinterpret_cast<const uint4 *>(xr + (grp + KS) * GROUP) + q);
+          for (int q = 0; q < 4; ++q) xn[q] = __ldg(reinterpret_cast<const uint4 *>(xr + (grp + KS) * GROUP) + q);
+        }
       }
       cp_async_wait<GV_DEPTH - 1>();  // group i's copies (this lane's) have landed
       const uint4 *sr = ring + (i % GV_DEPTH) * (4 * 32) + lane;
@@ -173,8 +180,6 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
       float pg[4] = {0.f, 0.f, 0.f, 0.f}, pu[4] = {0.f, 0.f, 0.f, 0.f};
       mma_group(pg, g0, g1, xb);
       mma_group(pu, u0, u1, xb);
-      const float sg0 = bf16_to_f(gs[grp]), sg1 = bf16_to_f(gs[8 * G + grp]);
-      const float su0 = bf16_to_f(us[grp]), su1 = bf16_to_f(us[8 * G + grp]);
       ag[0] = fmaf(sg0, pg[0], ag[0]); ag[1] = fmaf(sg0, pg[1], ag[1]);
       ag[2] = fmaf(sg1, pg[2], ag[2]); ag[3] = fmaf(sg1, pg[3], ag[3]);
       au[0] = fmaf(su0, pu[0], au[0]); au[1] = fmaf(su0, pu[1], au[1]);
