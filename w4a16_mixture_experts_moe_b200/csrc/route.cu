@@ -91,7 +91,6 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
   __shared__ float keys[MAX_E];                   // the token this CTA ranks
   cg::cluster_group cluster = cg::this_cluster();
   pdl_trigger();
-  pdl_wait();
   const int rank = int(cluster.block_rank());
   const int t0 = (blockIdx.x / RT_CLUSTER) * TOK;
   const int nt = min(TOK, T - t0);
@@ -99,21 +98,24 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
   const int EPC = (E + RT_CLUSTER - 1) / RT_CLUSTER;
   const int e_lo = rank * EPC, e_hi = min(E, e_lo + EPC);
   const bool given = flags & MOE_LOGITS_GIVEN;
+  // this warp's first router row: the router weights are not written by the
+  // preceding kernel, so these loads go out before waiting for it
+  constexpr int PRE = 8;
+  uint4 wpre[PRE];
+  const int e_first = e_lo + warp;
+  if (!given) {
+#pragma unroll
+    for (int u = 0; u < PRE; ++u) {
+      const int hc = lane + 32 * u;
+      wpre[u] = (e_first < e_hi && hc < H / 8) ? __ldg(reinterpret_cast<const uint4 *>(wr + int64_t(e_first) * H) + hc)
+                                              : make_uint4(0, 0, 0, 0);
+    }
+  }
+  pdl_wait();
 
   if (!given) {
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [TOK][H]
     const int chunks = H / 8;
-    // this warp's first router row: its loads go out before the activations'
-    // so the two round trips overlap
-    constexpr int PRE = 8;
-    uint4 wpre[PRE];
-    const int e_first = e_lo + warp;
-#pragma unroll
-    for (int u = 0; u < PRE; ++u) {
-      const int hc = lane + 32 * u;
-      wpre[u] = (e_first < e_hi && hc < chunks) ? __ldg(reinterpret_cast<const uint4 *>(wr + int64_t(e_first) * H) + hc)
-                                                 : make_uint4(0, 0, 0, 0);
-    }
     // the 8 tokens' rows, RT_THREADS 16-byte pieces per pass with all of a
     // batch's loads issued before any store (one round trip, not one per piece)
     constexpr int XB = 8;
