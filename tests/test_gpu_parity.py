@@ -215,7 +215,8 @@ def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None):
 
 @pytest.mark.parametrize("path", ["gemv", "tc"])
 @pytest.mark.parametrize("E,H,I,T,k", [(5, 256, 384, 13, 2), (4, 512, 256, 40, 3), (64, 2048, 1024, 16, 8),
-                                       (8, 4096, 1024, 9, 2), (4, 512, 256, 300, 2), (6, 384, 640, 700, 3)])
+                                       (8, 4096, 1024, 9, 2), (4, 512, 256, 300, 2), (6, 384, 640, 700, 3),
+                                       (64, 2048, 1024, 1, 8), (64, 2048, 1024, 64, 8)])
 def test_grouped_ffn(M, path, E, H, I, T, k):
     P = {"gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC}[path]
     rng = np.random.default_rng(E * H + T)
