@@ -14,7 +14,9 @@ e2e:    the same metric with the activations copied host->device from pinned
 roofline: the grouped FFN (gate/up + down kernels) per layer call: algorithmic
         bytes = active experts x 3,244,032 B of packed codes + scales, over the
         call's CUDA-event duration, against the measured HBM copy bandwidth.
-cpu_baseline: the CPU oracle (numpy, fp64) on a bounded sample of the workload.
+cpu_baseline: the CPU oracle (plain C, fp64, OpenMP over experts and tokens)
+        on a bounded sample of the workload: whole passes of layer 0 at the
+        bench's T, repeated for about ten seconds.
 
 --impl reference runs that oracle as the reference arm (rank 0 only).
 Multi-GPU: replicas only (each rank runs the whole workload on its own GPU;
@@ -313,42 +315,47 @@ def measure_T(stack, T, steps, warmup, world, want_e2e=True, want_roofline=True)
 
 # ----------------------------------------------------------------------------- CPU oracle (baseline / reference)
 
-def oracle_sample(T, reps):
-    """Time the oracle on `reps` passes of one OLMoE layer at T tokens.
-    Returns (layer-tokens per second, cores, description). Quantisation (an
-    offline step on both sides) is done before the clock starts."""
+def oracle_sample(T, seconds, shape="olmoe", tokens=None, skew=False, renorm=False, max_reps=200):
+    """Time the C oracle on whole passes of one layer of `shape` for about
+    `seconds` (at least one pass), on the first `tokens` of the T tokens
+    (all of them by default). Returns (layer-tokens per second, threads,
+    description). Quantisation (an offline step on both sides) is done before
+    the clock starts."""
     import numpy as np
     import torch
 
     import synth
-    from oracle import exactmoe_oracle as o
-    from threadpoolctl import threadpool_info
-    gate, up, down = synth.expert_bank(0, E, H, I, device="cuda" if torch.cuda.is_available() else "cpu")
-    g, u, d = gate.cpu(), up.cpu(), down.cpu()
-    del gate, up, down
-    packs = [[o.quantize_pack(m[e].double().numpy()) for e in range(E)] for m in (g, u, d)]
-    arrays = []
-    for m in packs:
-        arrays.append(np.stack([p for p, _ in m]))
-        arrays.append(np.stack([s for _, s in m]))
-    wr = synth.router_weight(0, E, H).double().numpy()
-    x = synth.activations(T, H).double().numpy()
+    from oracle import c_oracle as c
+    H_, I_, E_, K_ = SHAPES[shape]
+    Ts = T if tokens is None else min(T, tokens)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    mats = synth.expert_bank(0, E_, H_, I_, device=dev)
+    bits = [m.view(torch.int16).cpu().numpy().view(np.uint16) for m in mats]
+    del mats
+    packs = c.pack_experts(*bits, bits=True)
+    del bits
+    wr = synth.router_weight(0, E_, H_).double().numpy()
+    x = synth.activations(T, H_).double().numpy()[:Ts]
+    bias = synth.zipf_log_bias(E_) if skew else None
+    reps = 0
     t0 = time.perf_counter()
-    for _ in range(reps):
-        experts = o.PackedExperts(*arrays)       # fresh: dequantisation is part of the timed work
-        o.moe_layer(x, wr, experts, K, residual=x)
-    dt = time.perf_counter() - t0
-    cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    return T * reps / dt, cores, f"{reps} pass(es) of layer 0 of the stack at T={T} (dequant + router + top-k + " \
-                                 f"grouping + FFN + combine; quantisation not timed), {dt:.1f} s"
+    while True:
+        c.moe_layer(x, wr, packs, K_, bias, renorm, residual=True)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds or reps >= max_reps:
+            break
+    part = f"the first {Ts} of the T={T} tokens" if Ts < T else f"T={T}"
+    return Ts * reps / dt, c.threads(), f"{reps} pass(es) of layer 0 ({shape}) at {part} by the C oracle " \
+                                        f"(router + top-k + grouping + FFN with on-the-fly dequantisation + " \
+                                        f"combine; quantisation not timed), {dt:.1f} s"
 
 
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    reps = max(1, a.steps // 10)
-    v, cores, desc = oracle_sample(a.T, reps)
+    v, cores, desc = oracle_sample(a.T, seconds=min(60.0, 2.0 * max(1, a.steps)))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "layer-tokens/s", "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * a.T * a.layers / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -389,7 +396,7 @@ def main():
                              "n_active_mean": r["n_active_mean"]}
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        v, cores, desc = oracle_sample(a.T, 2)
+        v, cores, desc = oracle_sample(a.T, seconds=10.0)
         cpu = {"value": v, "unit": "layer-tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
     if world > 1:
         import torch.distributed as dist
@@ -536,6 +543,12 @@ def main_prefill(a, rank, world, P):
     H_, I_, E_, K_ = SHAPES[a.shape]
     stack = Stack(a.layers, a.path, a.shape, renorm=(a.shape == "wide"), skew=a.skew)
     r = measure_T(stack, a.T, a.steps, a.warmup, world)
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        del stack
+        v, cores, desc = oracle_sample(a.T, seconds=10.0, shape=a.shape, tokens=64, skew=a.skew,
+                                       renorm=(a.shape == "wide"))
+        cpu = {"value": v, "unit": "layer-tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
     if rank == 0:
         T, L = a.T, a.layers
         achieved = r["ffn_flops_per_call"] / (r["ffn_ms_per_call"] / 1e3) / 1e12
@@ -556,7 +569,7 @@ def main_prefill(a, rank, world, P):
                          "frac_of_sustained": achieved / P["bf16_tflops_sustained"], "traffic": None,
                          "peak_source": P["source"], "flops_per_call": r["ffn_flops_per_call"],
                          "ms_per_call": r["ffn_ms_per_call"], "n_active_mean": r["n_active_mean"]},
-            "cpu_baseline": None,
+            "cpu_baseline": cpu,
             "gpu_launches": r["launches_per_step"] * a.steps,
             "clocks": r["clocks"],
         }
