@@ -167,7 +167,7 @@ def test_slot_cache_decode_matches_resident(M):
     cache.close()
 
 
-@pytest.mark.parametrize("T", [512, 2048])
+@pytest.mark.parametrize("T", [512, 2048, 8192])
 def test_prefill_olmoe_tensor_core_sampled(M, T):
     """Prefill-sized OLMoE layer (AUTO picks the tcgen05 path: >= 32 rows per
     expert on average); every token is computed, a seeded sample is checked."""
@@ -183,10 +183,11 @@ def test_prefill_olmoe_tensor_core_sampled(M, T):
     _compare(out[sample], buf.topk_ids.cpu().numpy()[sample], ref, ref_ids, f"prefill T={T} sample")
 
 
-def test_prefill_second_shape_sampled(M):
-    """Hidden 4096, intermediate 14336, 8 experts, top-2 at T=512 (tcgen05 path)."""
+@pytest.mark.parametrize("T", [512, 8192])
+def test_prefill_second_shape_sampled(M, T):
+    """Hidden 4096, intermediate 14336, 8 experts, top-2 (tcgen05 path)."""
     from w4a16_mixture_experts_moe_b200.layer import ExpertBank, LayerBuffers, moe_layer_forward
-    H2, I2, E2, K2, T = 4096, 14336, 8, 2, 512
+    H2, I2, E2, K2 = 4096, 14336, 8, 2
     g, u, d = synth.expert_bank(0, E2, H2, I2)
     wr = synth.router_weight(0, E2, H2)
     bank = ExpertBank(E2, H2, I2)
@@ -199,4 +200,4 @@ def test_prefill_second_shape_sampled(M):
     sample = np.sort(np.random.default_rng(7).choice(T, size=12, replace=False))
     experts = o.LazyQuantizedExperts(torch_weights_source(g, u, d), E2, H2, I2, cache=1)
     ref, _, ref_ids, _ = o.moe_layer(x.double().numpy()[sample], wr.double().numpy(), experts, K2, renorm=True)
-    _compare(out[sample], buf.topk_ids.cpu().numpy()[sample], ref, ref_ids, "second shape T=512 sample")
+    _compare(out[sample], buf.topk_ids.cpu().numpy()[sample], ref, ref_ids, f"second shape T={T} sample")
