@@ -2,6 +2,7 @@
 gloo. The timing a rank reports is the max over ranks; the job's value counts
 every rank's units over that time; the reference arm runs on rank 0 alone."""
 import io
+import json
 import os
 import socket
 import sys
@@ -59,3 +60,27 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     with redirect_stdout(buf):
         bench.run_reference(a)
     assert buf.getvalue() == ""                       # the other ranks exit without work
+
+
+def test_reference_arm_line_on_rank_zero(monkeypatch):
+    # the oracle on a tiny stand-in shape, so the test stays fast: the line
+    # must carry the contract's keys, with the oracle as the CPU baseline and
+    # an e2e that moves no bytes
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setitem(bench.SHAPES, "olmoe", (256, 128, 4, 2))
+    monkeypatch.setattr(bench, "H", 256)
+    monkeypatch.setattr(bench, "I", 128)
+    monkeypatch.setattr(bench, "E", 4)
+    monkeypatch.setattr(bench, "K", 2)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3", "--T", "4"])
+    a = bench.parse()
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.run_reference(a)
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "layer-tokens/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["higher_is_better"] is True and line["steps"] == 1 and line["warmup"] == 3
