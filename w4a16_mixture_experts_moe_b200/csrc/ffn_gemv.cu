@@ -212,97 +212,109 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
   }
 }
 
-// down: y[r][row] = h[r] . Wd[row] (fp32), 16 output features per slice,
-// KS warps per slice as in the gate/up pass. A warp takes NS consecutive
-// slices and its ring streams straight through them: with four warps per
-// slice each walks only a quarter of K = I, so one slice alone would leave the
-// ring's start-up a large part of the CTA's life.
-template <int KS, int NS>
+// down: y[r][row] = h[r] . Wd[row] (fp32). A warp owns 32 output rows (two
+// 16-row slices side by side): per 128-wide group it copies 16 bytes of rows
+// g, g+8, g+16 and g+24 (2 KB per warp, as in the gate/up pass) and runs both
+// slices' MMAs on the same h fragment, which it loads one group ahead with
+// the group's scales. KS warps split the groups of a slice pair as in the
+// gate/up pass. (One 16-row slice per warp, half the bytes per h fragment,
+// measured 3-10 % slower.)
+template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs a) {
-  __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][4][32];
-  __shared__ uint4 rings[GV_WARPS][GV_DEPTH * 2 * 32];  // [slot][row g, row g+8][lane]
+  __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][8][32];
+  __shared__ uint4 rings[GV_WARPS][GV_DEPTH * 4 * 32];  // [slot][rows g, g+8, g+16, g+24][lane]
   pdl_trigger();
   pdl_wait();
   const int e = blockIdx.y;
   const int lo = a.offsets[e], cnt = a.offsets[e + 1] - lo;
   if (cnt <= 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int sl = warp / KS, kq = warp % KS;
-  const int row0 = (blockIdx.x * (GV_WARPS / KS) + sl) * NS * 16;  // first row of the warp's NS slices
-  if (blockIdx.x * (GV_WARPS / KS) * NS * 16 >= a.H) return;
+  const int sl = warp / KS, kq = warp % KS;  // slice pair within the CTA, K part
+  const int row0 = (blockIdx.x * (GV_WARPS / KS) + sl) * 32;
+  if (blockIdx.x * (GV_WARPS / KS) * 32 >= a.H) return;  // whole CTA out of range (uniform)
+  const bool rows_ok = row0 < a.H;  // H is a multiple of 128, so then all 32 rows are
   const uint8_t *rec = expert_record(a, e);
   if (!rec) return;
   const int I = a.I, KB = I / 2, G = I / GROUP;
-  const uint8_t *dq0 = rec + a.off_dq + int64_t(row0 + g) * KB + t * 16;
-  const uint16_t *ds = reinterpret_cast<const uint16_t *>(rec + a.off_ds) + int64_t(row0 + g) * G;
+  const int rr = rows_ok ? row0 + g : 0;
+  const uint8_t *dq0 = rec + a.off_dq + int64_t(rr) * KB + t * 16;
+  const uint16_t *ds = reinterpret_cast<const uint16_t *>(rec + a.off_ds) + int64_t(rr) * G;
 
   for (int n0 = 0; n0 < cnt; n0 += 8) {
     const bool ok = n0 + g < cnt;
     const uint16_t *hr = a.h + int64_t(lo + (ok ? n0 + g : 0)) * I + t * 32;
-    const int ngrp = kq < G ? (G - 1 - kq) / KS + 1 : 0;
-    // slices past the end of H get no positions
-    int ns = 0;
-#pragma unroll
-    for (int s = 0; s < NS; ++s) ns += row0 + s * 16 < a.H ? 1 : 0;
-    const int npos = ns * ngrp;
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    const int ngrp = rows_ok && kq < G ? (G - 1 - kq) / KS + 1 : 0;
     uint4 *ring = rings[warp];
-    auto issue = [&](int pos) {  // position = slice * ngrp + group ordinal
-      const int sc = pos / ngrp, grp = kq + (pos - sc * ngrp) * KS;
-      const uint8_t *src = dq0 + int64_t(sc) * 16 * KB + grp * 64;
-      uint4 *d = ring + (pos % GV_DEPTH) * (2 * 32) + lane;
-      cp_async16(d, src);
-      cp_async16(d + 32, src + 8 * KB);
+    auto issue = [&](int i) {
+      const int grp = kq + i * KS;
+      uint4 *d = ring + (i % GV_DEPTH) * (4 * 32) + lane;
+      cp_async16(d, dq0 + grp * 64);
+      cp_async16(d + 32, dq0 + 8 * KB + grp * 64);
+      cp_async16(d + 64, dq0 + 16 * KB + grp * 64);
+      cp_async16(d + 96, dq0 + 24 * KB + grp * 64);
     };
 #pragma unroll
     for (int i = 0; i < GV_DEPTH - 1; ++i) {
-      if (i < npos) issue(i);
+      if (i < ngrp) issue(i);
       cp_async_commit();
     }
-    int pos = 0;
-    for (int sc = 0; sc < NS; ++sc) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const bool slice_ok = sc < ns;
-      for (int i = 0; i < (slice_ok ? ngrp : 0); ++i, ++pos) {
-        const int grp = kq + i * KS;
-        if (pos + GV_DEPTH - 1 < npos) issue(pos + GV_DEPTH - 1);
-        cp_async_commit();
-        cp_async_wait<GV_DEPTH - 1>();  // this position's copies (this lane's) have landed
-        const uint4 *sr = ring + (pos % GV_DEPTH) * (2 * 32) + lane;
-        const uint4 w0 = sr[0], w1 = sr[32];
-        uint4 xb[4];
+    uint4 xn[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          xb[q] = ok ? *(reinterpret_cast<const uint4 *>(hr + grp * GROUP) + q) : make_uint4(0, 0, 0, 0);
-        float p[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_group(p, w0, w1, xb);
-        const uint16_t *dss = ds + int64_t(sc) * 16 * G;
-        const float s0 = bf16_to_f(dss[grp]), s1 = bf16_to_f(dss[8 * G + grp]);
-        acc[0] = fmaf(s0, p[0], acc[0]); acc[1] = fmaf(s0, p[1], acc[1]);
-        acc[2] = fmaf(s1, p[2], acc[2]); acc[3] = fmaf(s1, p[3], acc[3]);
+    for (int q = 0; q < 4; ++q)
+      xn[q] = ok && ngrp > 0 ? *(reinterpret_cast<const uint4 *>(hr + kq * GROUP) + q) : make_uint4(0, 0, 0, 0);
+    uint16_t s00 = 0, s01 = 0, s10 = 0, s11 = 0;  // scales of rows g, g+8 (slice 0) and g+16, g+24 (slice 1)
+    if (ngrp > 0) { s00 = ds[kq]; s01 = ds[8 * G + kq]; s10 = ds[16 * G + kq]; s11 = ds[24 * G + kq]; }
+    for (int i = 0; i < ngrp; ++i) {
+      const int grp = kq + i * KS;
+      if (i + GV_DEPTH - 1 < ngrp) issue(i + GV_DEPTH - 1);
+      cp_async_commit();
+      uint4 xb[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xb[q] = xn[q];
+      const float c00 = bf16_to_f(s00), c01 = bf16_to_f(s01), c10 = bf16_to_f(s10), c11 = bf16_to_f(s11);
+      if (i + 1 < ngrp) {
+        s00 = ds[grp + KS]; s01 = ds[8 * G + grp + KS]; s10 = ds[16 * G + grp + KS]; s11 = ds[24 * G + grp + KS];
+        if (ok) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) xn[q] = *(reinterpret_cast<const uint4 *>(hr + (grp + KS) * GROUP) + q);
+        }
       }
-      if (KS > 1) {
-        __syncthreads();
-        if (kq > 0) {
+      cp_async_wait<GV_DEPTH - 1>();  // group i's copies (this lane's) have landed
+      const uint4 *sr = ring + (i % GV_DEPTH) * (4 * 32) + lane;
+      const uint4 w0 = sr[0], w1 = sr[32], w2 = sr[64], w3 = sr[96];
+      float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_group(p0, w0, w1, xb);
+      mma_group(p1, w2, w3, xb);
+      a0[0] = fmaf(c00, p0[0], a0[0]); a0[1] = fmaf(c00, p0[1], a0[1]);
+      a0[2] = fmaf(c01, p0[2], a0[2]); a0[3] = fmaf(c01, p0[3], a0[3]);
+      a1[0] = fmaf(c10, p1[0], a1[0]); a1[1] = fmaf(c10, p1[1], a1[1]);
+      a1[2] = fmaf(c11, p1[2], a1[2]); a1[3] = fmaf(c11, p1[3], a1[3]);
+    }
+    if (KS > 1) {  // K parts 1.. hand their sums to part 0 of the slice pair
+      __syncthreads();
+      if (kq > 0) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) red[kq - 1][sl][c][lane] = acc[c];
-        }
-        __syncthreads();
-        if (kq == 0) {
-#pragma unroll
-          for (int q = 0; q < KS - 1; ++q)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[c] += red[q][sl][c][lane];
-        }
-        __syncthreads();  // `red` is reused by the next slice
+        for (int c = 0; c < 4; ++c) { red[kq - 1][sl][c][lane] = a0[c]; red[kq - 1][sl][4 + c][lane] = a1[c]; }
       }
+      __syncthreads();
+      if (kq == 0) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int r = n0 + 2 * t + c;
-        if (kq == 0 && slice_ok && r < cnt) {
-          float *yr = a.y + int64_t(lo + r) * a.H + row0 + sc * 16 + g;
-          yr[0] = acc[c];
-          yr[8] = acc[2 + c];
-        }
+        for (int q = 0; q < KS - 1; ++q)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) { a0[c] += red[q][sl][c][lane]; a1[c] += red[q][sl][4 + c][lane]; }
+      }
+    }
+    // accumulator (c0, c1) = row g, tokens 2t, 2t+1; (c2, c3) = row g+8
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int r = n0 + 2 * t + c;
+      if (kq == 0 && rows_ok && r < cnt) {
+        float *yr = a.y + int64_t(lo + r) * a.H + row0 + g;
+        yr[0] = a0[c];
+        yr[8] = a0[2 + c];
+        yr[16] = a1[c];
+        yr[24] = a1[2 + c];
       }
     }
   }
@@ -315,11 +327,8 @@ static cudaError_t launch_gemv_pair(const FfnArgs &a, cudaStream_t s) {
   cudaError_t e = launch_pdl(gemv_gateup_kernel<KS>, g1, dim3(GV_WARPS * 32), 0, s, a);
   if (e != cudaSuccess) return e;
   count_launches(1);
-  // two slices per warp when four warps share each (few experts active);
-  // measured a loss otherwise
-  constexpr int NS = KS == 4 ? 2 : 1;
-  dim3 g2((a.H + rows_per_cta * NS - 1) / (rows_per_cta * NS), a.E);
-  e = launch_pdl(gemv_down_kernel<KS, NS>, g2, dim3(GV_WARPS * 32), 0, s, a);
+  dim3 g2((a.H + rows_per_cta * 2 - 1) / (rows_per_cta * 2), a.E);  // two slices per warp
+  e = launch_pdl(gemv_down_kernel<KS>, g2, dim3(GV_WARPS * 32), 0, s, a);
   if (e == cudaSuccess) count_launches(1);
   return e;
 }
