@@ -1,40 +1,41 @@
 // A5 + A6, decode-sized groups: a weight-streaming grouped GEMV on the
 // warp-level tensor-core MMA (mma.sync m16n8k16, FP16 in, fp32 out).
 //
-// A warp owns 16 output rows of one expert and walks K one 128-wide
-// quantisation group at a time (four groups per loop trip, so the load
-// offsets fold into the instructions). Lane (g, t) = (lane/4, lane%4) loads
-// 16 bytes (32 codes) of rows g and g+8 per matrix: the group's four lanes
-// read 64 contiguous bytes of each row. The codes never leave registers: each
-// packed word turns into four FP16x2 code pairs (exact integers) used
-// directly as A fragments. Because a dot product does not depend on the order
-// of its K terms, lane t's fragment slots are bound to ITS OWN 32 consecutive
-// k of the group (not the PTX fragment's k order); the B fragment (the
-// token's activations, FP16 copies) is loaded with the same binding, so lane t
-// reads 64 contiguous bytes of each token row. The fp32 sum of q*x over one
+// A warp owns 32 output rows of one expert (two 16-row slices side by side)
+// and walks K one 128-wide quantisation group at a time. Lane (g, t) =
+// (lane/4, lane%4) copies 16 bytes (32 codes) of rows g, g+8, g+16 and g+24
+// per matrix: the group's four lanes read 64 contiguous bytes of each row.
+// The codes never leave registers once read: each packed word turns into four
+// FP16x2 code pairs (exact integers) used directly as A fragments. Because a
+// dot product does not depend on the order of its K terms, lane t's fragment
+// slots are bound to ITS OWN 32 consecutive k of the group (not the PTX
+// fragment's k order); the B fragment (the tokens' activations, FP16 copies,
+// or h in the down pass) is loaded with the same binding, so lane t reads 64
+// contiguous bytes of each token row, and one B fragment feeds every MMA tile
+// of the warp (four in gate/up, two in down). The fp32 sum of q*x over one
 // group is then multiplied by that row's group scale, so the dequantised
 // weight q*s is never rounded.
 //
-// The codes stream through a per-warp shared-memory ring of GV_DEPTH group
-// slots filled by cp.async, GV_DEPTH - 1 groups ahead of the math: the bytes
-// in flight per SM then do not depend on registers, and at the loaded HBM
-// latency they are what bounds a streaming kernel's bandwidth. Each lane
-// copies, and later reads back, only its own 16-byte pieces, so its own
-// cp.async waits suffice.
+// The codes stream through a per-warp shared-memory ring filled by cp.async,
+// DEPTH - 1 groups ahead of the math (gate/up: 4 KB slots, 2 deep; down: 2 KB
+// slots, 4 deep), while each group's B fragment and scales are loaded one
+// group ahead into registers. Each lane copies, and later reads back, only its
+// own 16-byte pieces, so its own cp.async waits suffice.
 //
-// Why FP16 operands: this kernel is bound by integer instructions spent
-// unpacking codes, and FP16's 10-bit mantissa lets a nibble sit at bits 4-7
-// of a half: one LOP3 yields (1024 + u) and another (1024 + 16u) for the next
-// code, with no shift. Codes and BF16 activations are exact in FP16 (the
-// activations while |x| <= 65504, which the FP16 copy of x checks).
+// Why FP16 operands: unpacking codes costs integer instructions, and FP16's
+// 10-bit mantissa lets a nibble sit at bits 4-7 of a half: one LOP3 yields
+// (1024 + u) and another (1024 + 16u) for the next code, with no shift. Codes
+// and BF16 activations are exact in FP16 (the activations while |x| <= 65504,
+// which the FP16 copy of x checks).
 #include <cmath>
 
 #include "ffn.cuh"
 
 namespace moe {
 
-constexpr int GV_WARPS = 4;  // 64 rows per CTA
-constexpr int GV_DEPTH = 4;  // groups of codes in flight per warp (shared-memory ring)
+constexpr int GV_WARPS = 4;  // per CTA: 128 rows, or 128 / KS with a K split
+constexpr int GV_DEPTH = 4;   // down: groups of codes in flight per warp (shared-memory ring, 2 KB each)
+constexpr int GV_DEPTH2 = 2;  // gate/up: the same (4 KB each)
 
 // 16-byte asynchronous copy global -> shared, cached in L2 only.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -102,25 +103,29 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint4 &w0, cons
   mma_word(acc, w0.w, w1.w, xb[3]);
 }
 
-// gate/up + SwiGLU: h[r][row] for the expert's rows r, 16 features per
-// slice. KS warps share a slice and split its groups (g % KS == the warp's
-// index within the slice) when there are few active experts; their partial
-// sums meet in shared memory. h is the BF16-rounded value stored as FP16
-// (exact), the down pass's B.
+// gate/up + SwiGLU: h[r][row] for the expert's rows r. A warp owns 32 rows
+// (two 16-row slices side by side) of both matrices: per 128-wide group it
+// copies 4 KB of codes (rows g, g+8, g+16, g+24 of gate and of up) and runs
+// four MMA tiles on one x fragment, which it loads one group ahead with the
+// group's eight scales. KS warps share a slice pair and split its groups
+// (group % KS == the warp's index) when there are few active experts; their
+// partial sums meet in shared memory. h is the BF16-rounded value stored as
+// FP16 (exact), the down pass's B. (One slice per warp with a 4-deep ring,
+// and two slices with a 3-deep ring, measured 2-8 % slower.)
 template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArgs a) {
-  __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][8][32];
-  __shared__ uint4 rings[GV_WARPS][GV_DEPTH * 4 * 32];  // [slot][gate g, gate g+8, up g, up g+8][lane]
+  __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][KS > 1 ? 16 : 1][32];
+  __shared__ uint4 rings[GV_WARPS][GV_DEPTH2 * 8 * 32];  // [slot][gate g, g+8, g+16, g+24, up ...][lane]
   pdl_trigger();
   pdl_wait();
   const int e = blockIdx.y;
   const int lo = a.offsets[e], cnt = a.offsets[e + 1] - lo;
   if (cnt <= 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int sl = warp / KS, kq = warp % KS;  // row slice within the CTA, K part
-  const int row0 = (blockIdx.x * (GV_WARPS / KS) + sl) * 16;
-  if (blockIdx.x * (GV_WARPS / KS) * 16 >= a.I) return;  // whole CTA out of range (uniform)
-  const bool rows_ok = row0 < a.I;
+  const int sl = warp / KS, kq = warp % KS;
+  const int row0 = (blockIdx.x * (GV_WARPS / KS) + sl) * 32;
+  if (blockIdx.x * (GV_WARPS / KS) * 32 >= a.I) return;
+  const bool rows_ok = row0 < a.I;  // I is a multiple of 128, so then all 32 rows are
   const uint8_t *rec = expert_record(a, e);
   if (!rec) return;
   const int H = a.H, KB = H / 2, G = H / GROUP;
@@ -134,79 +139,93 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
     const bool ok = n0 + g < cnt;
     const int token = ok ? a.sorted_pair[lo + n0 + g] / a.k : 0;
     const uint16_t *xr = a.x16 + int64_t(token) * H + t * 32;
-    float ag[4] = {0.f, 0.f, 0.f, 0.f}, au[4] = {0.f, 0.f, 0.f, 0.f};
+    float ag[2][4] = {}, au[2][4] = {};
     const int ngrp = rows_ok && kq < G ? (G - 1 - kq) / KS + 1 : 0;
     uint4 *ring = rings[warp];
     auto issue = [&](int i) {
       const int grp = kq + i * KS;
-      uint4 *d = ring + (i % GV_DEPTH) * (4 * 32) + lane;
-      cp_async16(d, gq0 + grp * 64);
-      cp_async16(d + 32, gq0 + 8 * KB + grp * 64);
-      cp_async16(d + 64, uq0 + grp * 64);
-      cp_async16(d + 96, uq0 + 8 * KB + grp * 64);
+      uint4 *d = ring + (i % GV_DEPTH2) * (8 * 32) + lane;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        cp_async16(d + 32 * r, gq0 + r * 8 * KB + grp * 64);
+        cp_async16(d + 128 + 32 * r, uq0 + r * 8 * KB + grp * 64);
+      }
     };
 #pragma unroll
-    for (int i = 0; i < GV_DEPTH - 1; ++i) {
+    for (int i = 0; i < GV_DEPTH2 - 1; ++i) {
       if (i < ngrp) issue(i);
       cp_async_commit();
     }
-    // the lane's activations one group ahead (registers; L2 latency hidden
-    // behind the current group's math)
     uint4 xn[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       xn[q] = ok && ngrp > 0 ? __ldg(reinterpret_cast<const uint4 *>(xr + kq * GROUP) + q) : make_uint4(0, 0, 0, 0);
-    // the group's four scales, also one group ahead
-    uint16_t sgn0 = 0, sgn1 = 0, sun0 = 0, sun1 = 0;
-    if (ngrp > 0) { sgn0 = gs[kq]; sgn1 = gs[8 * G + kq]; sun0 = us[kq]; sun1 = us[8 * G + kq]; }
+    uint32_t sgn[2] = {0, 0}, sun[2] = {0, 0};  // BF16 scale pairs: rows (g, g+8), (g+16, g+24)
+    auto load_s = [&](int grp) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        sgn[h] = uint32_t(gs[16 * h * G + grp]) | (uint32_t(gs[(16 * h + 8) * G + grp]) << 16);
+        sun[h] = uint32_t(us[16 * h * G + grp]) | (uint32_t(us[(16 * h + 8) * G + grp]) << 16);
+      }
+    };
+    if (ngrp > 0) load_s(kq);
     for (int i = 0; i < ngrp; ++i) {
       const int grp = kq + i * KS;
-      if (i + GV_DEPTH - 1 < ngrp) issue(i + GV_DEPTH - 1);
+      if (i + GV_DEPTH2 - 1 < ngrp) issue(i + GV_DEPTH2 - 1);
       cp_async_commit();
       uint4 xb[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) xb[q] = xn[q];
-      const float sg0 = bf16_to_f(sgn0), sg1 = bf16_to_f(sgn1), su0 = bf16_to_f(sun0), su1 = bf16_to_f(sun1);
+      const uint32_t sg[2] = {sgn[0], sgn[1]}, su[2] = {sun[0], sun[1]};
       if (i + 1 < ngrp) {
-        sgn0 = gs[grp + KS]; sgn1 = gs[8 * G + grp + KS]; sun0 = us[grp + KS]; sun1 = us[8 * G + grp + KS];
+        load_s(grp + KS);
         if (ok) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) xn[q] = __ldg(reinterpret_cast<const uint4 *>(xr + (grp + KS) * GROUP) + q);
         }
       }
-      cp_async_wait<GV_DEPTH - 1>();  // group i's copies (this lane's) have landed
-      const uint4 *sr = ring + (i % GV_DEPTH) * (4 * 32) + lane;
-      const uint4 g0 = sr[0], g1 = sr[32], u0 = sr[64], u1 = sr[96];
-      float pg[4] = {0.f, 0.f, 0.f, 0.f}, pu[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_group(pg, g0, g1, xb);
-      mma_group(pu, u0, u1, xb);
-      ag[0] = fmaf(sg0, pg[0], ag[0]); ag[1] = fmaf(sg0, pg[1], ag[1]);
-      ag[2] = fmaf(sg1, pg[2], ag[2]); ag[3] = fmaf(sg1, pg[3], ag[3]);
-      au[0] = fmaf(su0, pu[0], au[0]); au[1] = fmaf(su0, pu[1], au[1]);
-      au[2] = fmaf(su1, pu[2], au[2]); au[3] = fmaf(su1, pu[3], au[3]);
+      cp_async_wait<GV_DEPTH2 - 1>();  // group i's copies (this lane's) have landed
+      const uint4 *sr = ring + (i % GV_DEPTH2) * (8 * 32) + lane;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float pg[4] = {0.f, 0.f, 0.f, 0.f}, pu[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_group(pg, sr[64 * h], sr[64 * h + 32], xb);
+        mma_group(pu, sr[128 + 64 * h], sr[128 + 64 * h + 32], xb);
+        const float g0 = bf16_lo(sg[h]), g1 = bf16_hi(sg[h]), u0 = bf16_lo(su[h]), u1 = bf16_hi(su[h]);
+        ag[h][0] = fmaf(g0, pg[0], ag[h][0]); ag[h][1] = fmaf(g0, pg[1], ag[h][1]);
+        ag[h][2] = fmaf(g1, pg[2], ag[h][2]); ag[h][3] = fmaf(g1, pg[3], ag[h][3]);
+        au[h][0] = fmaf(u0, pu[0], au[h][0]); au[h][1] = fmaf(u0, pu[1], au[h][1]);
+        au[h][2] = fmaf(u1, pu[2], au[h][2]); au[h][3] = fmaf(u1, pu[3], au[h][3]);
+      }
     }
-    if (KS > 1) {  // K parts 1.. hand their sums to part 0 of the slice
+    if (KS > 1) {
       __syncthreads();
       if (kq > 0) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) { red[kq - 1][sl][c][lane] = ag[c]; red[kq - 1][sl][4 + c][lane] = au[c]; }
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) { red[kq - 1][sl][8 * h + c][lane] = ag[h][c]; red[kq - 1][sl][8 * h + 4 + c][lane] = au[h][c]; }
       }
       __syncthreads();
       if (kq == 0) {
 #pragma unroll
         for (int q = 0; q < KS - 1; ++q)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) { ag[c] += red[q][sl][c][lane]; au[c] += red[q][sl][4 + c][lane]; }
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) { ag[h][c] += red[q][sl][8 * h + c][lane]; au[h][c] += red[q][sl][8 * h + 4 + c][lane]; }
       }
     }
-    // accumulator (c0, c1) = row g, tokens 2t, 2t+1; (c2, c3) = row g+8
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int r = n0 + 2 * t + c;
       if (kq == 0 && rows_ok && r < cnt) {
         uint16_t *hr = a.h + int64_t(lo + r) * a.I + row0 + g;
-        hr[0] = __half_as_ushort(__float2half_rn(bf16_to_f(f_to_bf16(silu_f(ag[c]) * au[c]))));
-        hr[8] = __half_as_ushort(__float2half_rn(bf16_to_f(f_to_bf16(silu_f(ag[2 + c]) * au[2 + c]))));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          hr[16 * h] = __half_as_ushort(__float2half_rn(bf16_to_f(f_to_bf16(silu_f(ag[h][c]) * au[h][c]))));
+          hr[16 * h + 8] = __half_as_ushort(__float2half_rn(bf16_to_f(f_to_bf16(silu_f(ag[h][2 + c]) * au[h][2 + c]))));
+        }
       }
     }
   }
@@ -323,7 +342,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
 template <int KS>
 static cudaError_t launch_gemv_pair(const FfnArgs &a, cudaStream_t s) {
   const int rows_per_cta = (GV_WARPS / KS) * 16;
-  dim3 g1((a.I + rows_per_cta - 1) / rows_per_cta, a.E);
+  dim3 g1((a.I + rows_per_cta * 2 - 1) / (rows_per_cta * 2), a.E);  // two slices per warp
   cudaError_t e = launch_pdl(gemv_gateup_kernel<KS>, g1, dim3(GV_WARPS * 32), 0, s, a);
   if (e != cudaSuccess) return e;
   count_launches(1);
