@@ -352,15 +352,17 @@ static cudaError_t launch_gemv_pair(const FfnArgs &a, cudaStream_t s) {
   return e;
 }
 
-// Warps that share a 16-row slice, from the expected number of active experts
-// E (1 - (1 - k/E)^T): enough warps to keep every SM streaming when a decode
-// step touches few experts (same-box measurements on the OLMoE decode stack
-// chose the thresholds).
+// Warps that share a 32-row slice pair, from the expected number of active
+// experts E (1 - (1 - k/E)^T): enough warps to keep every SM streaming when a
+// decode step touches few experts (same-box measurements on the OLMoE decode
+// stack chose the thresholds; at T = 16 two warps per pair gave the same FFN
+// time as one but a 2 us shorter layer step, the FFN overlapping its
+// neighbours better).
 static int pick_ksplit(const FfnArgs &a) {
   const double miss = 1.0 - double(a.k) / double(a.E);
   double n_act = double(a.E) * (1.0 - std::pow(miss, double(a.T)));
   if (n_act < 1.0) n_act = 1.0;
-  const double warps = n_act * (a.I / 16);
+  const double warps = n_act * (a.I / 32);  // one warp per slice pair of every active expert
   const double want = 148.0 * 24.0;
   // with 4+ rows per expert on average (several token chunks per CTA) two
   // warps per slice shorten each CTA's life enough to pay for the reduction
