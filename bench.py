@@ -42,11 +42,11 @@ SHAPES = {"olmoe": (2048, 1024, 64, 8), "wide": (4096, 14336, 8, 2)}   # (H, I, 
 
 # DRAM bytes (read + write) of one decode FFN call per active expert, from one
 # ncu capture of the gate/up and down GEMV launches at T=16 (57 active
-# experts; gate/up 119.04 MB read + 4.28 MB written, down 59.75 MB read +
-# 0.91 MB written).
+# experts; gate/up 119.04 MB read + 3.30 MB written, down 59.75 MB read +
+# 0.02 MB written).
 # Reported as roofline.traffic scaled to the bench's active experts; valid
 # while those kernels are the ones captured.
-DECODE_TRAFFIC_PER_ACTIVE_EXPERT = (119.037e6 + 4.283e6 + 59.746e6 + 0.911e6) / 57
+DECODE_TRAFFIC_PER_ACTIVE_EXPERT = (119.036e6 + 3.302e6 + 59.748e6 + 0.022e6) / 57
 
 
 def rec_bytes(h, i):
