@@ -34,8 +34,8 @@
 namespace moe {
 
 constexpr int GV_WARPS = 4;  // per CTA: 128 rows, or 128 / KS with a K split
-constexpr int GV_DEPTH = 4;   // down: groups of codes in flight per warp (shared-memory ring, 2 KB each)
-constexpr int GV_DEPTH2 = 2;  // gate/up: the same (4 KB each)
+constexpr int GV_DEPTH_DOWN = 4;    // down: ring slots (groups of codes) per warp, 2 KB each
+constexpr int GV_DEPTH_GATEUP = 2;  // gate/up: ring slots per warp, 4 KB each
 
 // 16-byte asynchronous copy global -> shared, cached in L2 only.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -115,7 +115,7 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint4 &w0, cons
 template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArgs a) {
   __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][KS > 1 ? 16 : 1][32];
-  __shared__ uint4 rings[GV_WARPS][GV_DEPTH2 * 8 * 32];  // [slot][gate g, g+8, g+16, g+24, up ...][lane]
+  __shared__ uint4 rings[GV_WARPS][GV_DEPTH_GATEUP * 8 * 32];  // [slot][gate g, g+8, g+16, g+24, up ...][lane]
   pdl_trigger();
   pdl_wait();
   const int e = blockIdx.y;
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
     uint4 *ring = rings[warp];
     auto issue = [&](int i) {
       const int grp = kq + i * KS;
-      uint4 *d = ring + (i % GV_DEPTH2) * (8 * 32) + lane;
+      uint4 *d = ring + (i % GV_DEPTH_GATEUP) * (8 * 32) + lane;
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         cp_async16(d + 32 * r, gq0 + r * 8 * KB + grp * 64);
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
       }
     };
 #pragma unroll
-    for (int i = 0; i < GV_DEPTH2 - 1; ++i) {
+    for (int i = 0; i < GV_DEPTH_GATEUP - 1; ++i) {
       if (i < ngrp) issue(i);
       cp_async_commit();
     }
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
     if (ngrp > 0) load_s(kq);
     for (int i = 0; i < ngrp; ++i) {
       const int grp = kq + i * KS;
-      if (i + GV_DEPTH2 - 1 < ngrp) issue(i + GV_DEPTH2 - 1);
+      if (i + GV_DEPTH_GATEUP - 1 < ngrp) issue(i + GV_DEPTH_GATEUP - 1);
       cp_async_commit();
       uint4 xb[4];
 #pragma unroll
@@ -184,8 +184,8 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
           for (int q = 0; q < 4; ++q) xn[q] = __ldg(reinterpret_cast<const uint4 *>(xr + (grp + KS) * GROUP) + q);
         }
       }
-      cp_async_wait<GV_DEPTH2 - 1>();  // group i's copies (this lane's) have landed
-      const uint4 *sr = ring + (i % GV_DEPTH2) * (8 * 32) + lane;
+      cp_async_wait<GV_DEPTH_GATEUP - 1>();  // group i's copies (this lane's) have landed
+      const uint4 *sr = ring + (i % GV_DEPTH_GATEUP) * (8 * 32) + lane;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float pg[4] = {0.f, 0.f, 0.f, 0.f}, pu[4] = {0.f, 0.f, 0.f, 0.f};
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
 template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs a) {
   __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][8][32];
-  __shared__ uint4 rings[GV_WARPS][GV_DEPTH * 4 * 32];  // [slot][rows g, g+8, g+16, g+24][lane]
+  __shared__ uint4 rings[GV_WARPS][GV_DEPTH_DOWN * 4 * 32];  // [slot][rows g, g+8, g+16, g+24][lane]
   pdl_trigger();
   pdl_wait();
   const int e = blockIdx.y;
@@ -267,14 +267,14 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
     uint4 *ring = rings[warp];
     auto issue = [&](int i) {
       const int grp = kq + i * KS;
-      uint4 *d = ring + (i % GV_DEPTH) * (4 * 32) + lane;
+      uint4 *d = ring + (i % GV_DEPTH_DOWN) * (4 * 32) + lane;
       cp_async16(d, dq0 + grp * 64);
       cp_async16(d + 32, dq0 + 8 * KB + grp * 64);
       cp_async16(d + 64, dq0 + 16 * KB + grp * 64);
       cp_async16(d + 96, dq0 + 24 * KB + grp * 64);
     };
 #pragma unroll
-    for (int i = 0; i < GV_DEPTH - 1; ++i) {
+    for (int i = 0; i < GV_DEPTH_DOWN - 1; ++i) {
       if (i < ngrp) issue(i);
       cp_async_commit();
     }
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
     if (ngrp > 0) { s00 = ds[kq]; s01 = ds[8 * G + kq]; s10 = ds[16 * G + kq]; s11 = ds[24 * G + kq]; }
     for (int i = 0; i < ngrp; ++i) {
       const int grp = kq + i * KS;
-      if (i + GV_DEPTH - 1 < ngrp) issue(i + GV_DEPTH - 1);
+      if (i + GV_DEPTH_DOWN - 1 < ngrp) issue(i + GV_DEPTH_DOWN - 1);
       cp_async_commit();
       uint4 xb[4];
 #pragma unroll
@@ -299,8 +299,8 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
           for (int q = 0; q < 4; ++q) xn[q] = *(reinterpret_cast<const uint4 *>(hr + (grp + KS) * GROUP) + q);
         }
       }
-      cp_async_wait<GV_DEPTH - 1>();  // group i's copies (this lane's) have landed
-      const uint4 *sr = ring + (i % GV_DEPTH) * (4 * 32) + lane;
+      cp_async_wait<GV_DEPTH_DOWN - 1>();  // group i's copies (this lane's) have landed
+      const uint4 *sr = ring + (i % GV_DEPTH_DOWN) * (4 * 32) + lane;
       const uint4 w0 = sr[0], w1 = sr[32], w2 = sr[64], w3 = sr[96];
       float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
       mma_group(p0, w0, w1, xb);
