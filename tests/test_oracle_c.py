@@ -233,3 +233,55 @@ def test_c_and_numpy_oracles_agree(T, E, H, I, k, renorm):
     oc = c.combine(yn, w_n, gn[3], x)
     on = o.combine(yn, w_n, gn[3], x)
     assert np.array_equal(oc, on)
+
+
+# ---------------------------------------------------------------- property checks (hypothesis)
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=30, deadline=None)
+@given(T=st.integers(0, 12), E=st.integers(1, 40), k=st.integers(1, 8), seed=st.integers(0, 2**31 - 1),
+       renorm=st.booleans(), biased=st.booleans())
+def test_property_routing_and_grouping_agree(T, E, k, seed, renorm, biased):
+    k = min(k, E)
+    rng = np.random.default_rng(seed)
+    logits = c.from_bits(c.to_bits(rng.standard_normal((T, E))))
+    if T and rng.random() < 0.3:
+        logits[0, :] = logits[0, 0]                       # a fully tied row
+    bias = (rng.standard_normal(E) * 0.3).astype(np.float32) if biased else None
+    ic, wc = c.route_topk(logits, k, bias, renorm)
+    i_n, w_n = o.route_topk(logits, k, bias, renorm)
+    assert np.array_equal(ic, i_n)
+    assert np.allclose(wc, w_n, rtol=1e-12, atol=0)
+    for a, b in zip(c.group_tokens(ic, E), o.group_tokens(i_n, E)):
+        assert np.array_equal(a, b)
+
+
+@settings(max_examples=20, deadline=None)
+@given(T=st.integers(1, 6), k=st.integers(1, 4), H=st.sampled_from([8, 64]), seed=st.integers(0, 2**31 - 1),
+       res=st.booleans(), drop=st.booleans())
+def test_property_combine_agrees(T, k, H, seed, res, drop):
+    rng = np.random.default_rng(seed)
+    y = rng.standard_normal((T * k, H))
+    w = rng.random((T, k))
+    pos = rng.permutation(T * k).astype(np.int32)
+    if drop:
+        pos[rng.integers(0, T * k)] = -1
+    r = c.from_bits(c.to_bits(rng.standard_normal((T, H)))) if res else None
+    assert np.array_equal(c.combine(y, w, pos, r), o.combine(y, w, pos, r))
+
+
+@settings(max_examples=12, deadline=None)
+@given(N=st.integers(1, 6), G=st.integers(1, 3), scale=st.sampled_from([1e-3, 0.02, 1.0, 300.0]),
+       seed=st.integers(0, 2**31 - 1))
+def test_property_quantiser_agrees_and_round_trips(N, G, scale, seed):
+    rng = np.random.default_rng(seed)
+    w = c.from_bits(c.to_bits(rng.standard_normal((N, 128 * G)) * scale))
+    if rng.random() < 0.3:
+        w[0, :128] = 0.0                                   # an all-zero group
+    pc, sc_ = c.quantize_pack(w)
+    pn, sn = o.quantize_pack(w)
+    assert np.array_equal(pc, pn) and np.array_equal(sc_, sn)
+    s = np.repeat(c.from_bits(sc_), 128, axis=1)
+    assert np.all(np.abs(w - c.dequantize_packed(pc, sc_)) <= s / 2 * (1 + 2.0 ** -20))
