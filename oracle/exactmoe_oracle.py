@@ -380,3 +380,103 @@ def moe_layer(x, w_router, experts: PackedExperts, k: int, bias=None,
     logits = router_logits(x, w_router)
     ids, w = route_topk(logits, k, bias, renorm)
     return moe_layer_grouped(x, experts, ids, w, residual), logits, ids, w
+
+
+# --------------------------------------------------------------------------
+# Expert slot cache (Abstract: a configurable GPU-resident slot cache over
+# experts kept in pinned host memory; Figure 1 caption: a miss moves the
+# packed weights and scales of the expert; Figure 2 caption: when the cache
+# holds every expert, lookup accounting is bypassed; Table 1: hit rate and
+# host-to-device traffic per slot count)
+# --------------------------------------------------------------------------
+
+class SlotCapacityError(ValueError):
+    """A step needs more distinct experts than the cache has slots."""
+
+
+class SlotCacheLRU:
+    """Policy of one layer's slot cache, as plain bookkeeping.
+
+    The pages name the cache and its counters but no replacement policy; the
+    reading used here is least-recently-used:
+
+    * a step's ids are de-duplicated (an expert chosen by several tokens of
+      the step is one lookup) and handled in first-occurrence order;
+    * an id already in a slot is a hit, and that slot counts as used by this
+      step;
+    * every other id is a miss: it takes the lowest-numbered empty slot if
+      one exists, otherwise it evicts the expert whose slot was used least
+      recently, never one used by this step, the lower slot number breaking
+      ties; a miss is one whole expert record copied host -> device;
+    * more distinct ids than slots is an error and changes nothing;
+    * with at least as many slots as experts the cache is resident: expert e
+      lives in slot e, the first use of an expert loads it, and hits and
+      misses are not counted.
+
+    `lookup` returns (slot of each id in the order given, ids loaded this
+    step, experts evicted this step).
+    """
+
+    def __init__(self, E: int, slots: int):
+        self.E, self.S = int(E), int(slots)
+        self.resident = self.S >= self.E
+        self.expert_in = [None] * self.S      # slot -> expert held
+        self.last_use = [0] * self.S          # slot -> step that last used it
+        self.step = 0
+        self.hits = self.misses = self.loads = 0
+
+    def slot_of(self, e: int):
+        if self.resident:
+            return e if self.expert_in[e] is not None else None
+        for s in range(self.S):
+            if self.expert_in[s] == e:
+                return s
+        return None
+
+    def lookup(self, ids):
+        ids = [int(v) for v in ids]
+        if any(v < 0 or v >= self.E for v in ids):
+            raise ValueError("expert id out of range")
+        distinct = []
+        for v in ids:
+            if v not in distinct:
+                distinct.append(v)
+        if len(distinct) > self.S:
+            raise SlotCapacityError(f"{len(distinct)} distinct experts > {self.S} slots")
+        self.step += 1
+        loaded, evicted = [], []
+        if self.resident:
+            for v in distinct:
+                if self.expert_in[v] is None:
+                    self.expert_in[v] = v
+                    loaded.append(v)
+            self.loads += len(loaded)
+            return [v for v in ids], loaded, evicted
+        in_use = set()
+        for v in distinct:                      # hits first: their slots are protected
+            s = self.slot_of(v)
+            if s is not None:
+                self.hits += 1
+                self.last_use[s] = self.step
+                in_use.add(s)
+        for v in distinct:
+            if self.slot_of(v) is not None:
+                continue
+            empty = [s for s in range(self.S) if self.expert_in[s] is None]
+            if empty:
+                s = empty[0]
+            else:
+                free = [s for s in range(self.S) if s not in in_use]
+                s = min(free, key=lambda c: (self.last_use[c], c))
+                evicted.append(self.expert_in[s])
+            self.expert_in[s] = v
+            self.last_use[s] = self.step
+            in_use.add(s)
+            self.misses += 1
+            self.loads += 1
+            loaded.append(v)
+        return [self.slot_of(v) for v in ids], loaded, evicted
+
+    def h2d_bytes(self, record_bytes: int) -> int:
+        """Host-to-device bytes moved so far: one record per load."""
+        return self.loads * int(record_bytes)

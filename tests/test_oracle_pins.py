@@ -138,6 +138,44 @@ def test_router_logits_match_library_matmul():
     assert np.array_equal(got, ref)
 
 
+def test_router_logits_hand_computed():
+    # integer-valued operands make every product and sum exact, so the values
+    # below are worked by hand; E = 3 and H = 4 differ, so a transposed router
+    # fails on shape, and each row of W picks out a different combination of x
+    x = np.array([[1.0, -2.0, 3.0, 0.5],
+                  [0.0, 1.0, 1.0, 1.0]])
+    wr = np.array([[1.0, 1.0, 1.0, 1.0],       # sum of x
+                   [2.0, 0.0, -1.0, 4.0],      # 2*x0 - x2 + 4*x3
+                   [0.25, 0.0, 0.0, -8.0]])    # x0/4 - 8*x3
+    want = np.array([[2.5, 1.0, -3.75],
+                     [3.0, 3.0, -8.0]])
+    assert np.array_equal(o.router_logits(x, wr), want)
+    # the one rounding to BF16 (8 significant bits), ties to even: 257 and 259
+    # lie halfway between neighbours 2 apart and go to 256 and 260; 257.5 is
+    # just above the midpoint and goes to 258
+    ones = np.ones((3, 1))
+    xs = np.array([[257.0], [259.0], [257.5]])
+    assert list(o.router_logits(xs, ones)[:, 0]) == [256.0, 260.0, 258.0]
+
+
+def test_weights_for_given_ids():
+    # probabilities of given ids are the full softmax at those ids, in the
+    # order given (scipy); for the top-k ids they equal route_topk's weights;
+    # renormalised ones sum to one
+    rng = np.random.default_rng(9)
+    T, E, k = 6, 10, 3
+    logits = o.round_to_bf16(rng.standard_normal((T, E)))
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
+    p = scipy.special.softmax(logits, axis=1)
+    w = o.weights_for_ids(logits, ids)
+    assert np.allclose(w, np.take_along_axis(p, ids, axis=1), rtol=1e-14, atol=0)
+    wn = o.weights_for_ids(logits, ids, renorm=True)
+    assert np.allclose(wn.sum(axis=1), 1.0, rtol=1e-14)
+    assert np.allclose(wn, w / w.sum(axis=1, keepdims=True), rtol=1e-14)
+    top, wt = o.route_topk(logits, k)
+    assert np.array_equal(o.weights_for_ids(logits, top), wt)
+
+
 def _brute_topk(key_row, k):
     E = len(key_row)
     keyv = [(-np.inf if np.isnan(v) else float(v)) for v in key_row]
@@ -275,3 +313,85 @@ def test_combine_dropped_pair_equals_zero_weight():
     w0[2, 1] = 0.0
     assert np.array_equal(o.combine(y, w, dropped, res), o.combine(y, w0, pos, res))
 
+
+
+# ---------------------------------------------------------------- slot cache (A8)
+
+LRU_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "slot_cache_lru_trace.json")
+
+
+def test_slot_cache_hand_worked_trace():
+    g = json.load(open(LRU_GOLDEN))
+    c = o.SlotCacheLRU(g["E"], g["slots"])
+    for st in g["steps"]:
+        if st.get("capacity_error"):
+            with pytest.raises(o.SlotCapacityError):
+                c.lookup(st["ids"])
+        else:
+            slots, loaded, evicted = c.lookup(st["ids"])
+            assert slots == st["slot_of_ids"], st
+            assert loaded == st["loaded"], st
+            assert evicted == st["evicted"], st
+        assert (c.hits, c.misses) == (st["hits"], st["misses"]), st
+    r = g["resident"]
+    c = o.SlotCacheLRU(r["E"], r["slots"])
+    for st in r["steps"]:
+        slots, loaded, evicted = c.lookup(st["ids"])
+        assert (slots, loaded, evicted) == (st["slot_of_ids"], st["loaded"], [])
+    assert (c.hits, c.misses, c.loads) == (r["hits"], r["misses"], r["loads"])
+    assert c.h2d_bytes(1000) == 1000 * r["loads"]
+
+
+@pytest.mark.parametrize("S", [1, 2, 3, 5, 8])
+def test_slot_cache_one_id_per_step_equals_library_lru(S):
+    # with one expert per step the policy is a plain LRU cache of S entries:
+    # its hit count equals that of functools.lru_cache(maxsize=S) on the
+    # same sequence of keys
+    import functools
+    rng = np.random.default_rng(S)
+    seq = [int(v) for v in rng.integers(0, 9, size=400)]
+
+    @functools.lru_cache(maxsize=S)
+    def touch(e):
+        return e
+
+    c = o.SlotCacheLRU(9, S)
+    for e in seq:
+        touch(e)
+        c.lookup([e])
+    info = touch.cache_info()
+    assert (c.hits, c.misses) == (info.hits, info.misses)
+
+
+def test_slot_cache_cyclic_sweep_never_hits_and_invariants_hold():
+    # a cyclic sweep over S + 1 experts defeats LRU completely (each expert
+    # is evicted just before it comes back); S experts fit and always hit
+    S = 4
+    c = o.SlotCacheLRU(16, S)
+    for r in range(5):
+        for e in range(S + 1):
+            c.lookup([e])
+    assert c.hits == 0 and c.misses == 5 * (S + 1)
+    c = o.SlotCacheLRU(16, S)
+    for r in range(5):
+        c.lookup(list(range(S)))
+    assert (c.hits, c.misses) == (4 * S, S)
+    # random multi-id steps: every id is held afterwards in distinct slots, an
+    # evicted expert was not needed by the step, and the counters add up
+    rng = np.random.default_rng(3)
+    c = o.SlotCacheLRU(12, 5)
+    lookups = 0
+    for _ in range(300):
+        ids = [int(v) for v in rng.integers(0, 12, size=rng.integers(1, 7))]
+        if len(set(ids)) > 5:
+            with pytest.raises(o.SlotCapacityError):
+                c.lookup(ids)
+            continue
+        slots, loaded, evicted = c.lookup(ids)
+        lookups += len(set(ids))
+        held = {e: c.slot_of(e) for e in set(ids)}
+        assert all(held[e] == s for e, s in zip(ids, slots))
+        assert len(set(held.values())) == len(held)
+        assert not set(evicted) & set(ids)
+        assert set(loaded) <= set(ids)
+    assert c.hits + c.misses == lookups
