@@ -74,84 +74,50 @@ def test_argument_checks_run_before_any_cuda_call(native):
     assert lib.moe_route_topk(None, None, 0, 2048, 64, 8, None, 0, None, None, None, None) == native.MOE_OK
 
 
-class _LRUModel:
-    """Plain model of the slot cache policy for the host tests."""
-
-    def __init__(self, E, S):
-        self.E, self.S = E, S
-        self.owner = [-1] * S
-        self.stamp = [0] * S
-        self.where = {}
-        self.now = 0
-        self.hits = self.misses = 0
-
-    def lookup(self, ids):
-        self.now += 1
-        uniq = list(dict.fromkeys(ids))
-        miss = []
-        for e in uniq:
-            if e in self.where:
-                self.stamp[self.where[e]] = self.now
-                self.hits += 1
-            else:
-                miss.append(e)
-        for e in miss:
-            free = [s for s in range(self.S) if self.stamp[s] != self.now and self.owner[s] < 0]
-            if free:
-                v = free[0]
-            else:
-                cands = [s for s in range(self.S) if self.stamp[s] != self.now]
-                v = min(cands, key=lambda s: (self.stamp[s], s))
-            if self.owner[v] >= 0:
-                del self.where[self.owner[v]]
-            self.owner[v] = e
-            self.where[e] = v
-            self.stamp[v] = self.now
-            self.misses += 1
-        return [self.where[e] for e in ids], miss
-
-
-def test_slot_cache_lru_matches_model(native):
-    import numpy as np
+def test_slot_cache_lru_matches_oracle(native):
+    """The library's host LRU against the oracle's slot-cache policy."""
     import synth
+    from oracle import exactmoe_oracle as o
     E, S, k, steps = 64, 16, 8, 200
-    c = native.SlotCache(1, E, S, 256, 0x1000, 0x2000, 0x3000)   # fake addresses: lookups never dereference
-    model = _LRUModel(E, S)
+    c = native.SlotCache(1, E, S, 256, None, None, None)   # no memory: simulates the policy
+    model = o.SlotCacheLRU(E, S)
     routing = synth.drawn_routing(0, E, k, steps)
     for s in range(steps):
         ids = [int(v) for v in routing[s]]
         got = c.lookup(0, ids)
-        want = model.lookup(ids)
-        assert got == want, s
+        slots, loaded, _ = model.lookup(ids)
+        assert got == (slots, loaded), s
+        c.fill(0, got[1], side=0, compute=0)         # simulated: counts the copies
         # every id maps to a distinct slot this step
         assert len(set(got[0])) == len(ids)
     st = c.stats()
     assert (st["hits"], st["misses"]) == (model.hits, model.misses)
-    assert st["h2d_bytes"] == 0      # no fill was issued
+    assert st["h2d_bytes"] == model.h2d_bytes(256)
     # keep-probability 0.5 routing over 16 slots: a fair share of hits
     assert 0.3 < st["hits"] / (st["hits"] + st["misses"]) < 0.9
     c.close()
 
 
 def test_slot_cache_capacity_duplicates_and_resident_mode(native):
-    c = native.SlotCache(2, 8, 2, 256, 0x1000, 0x2000, 0x3000)
+    c = native.SlotCache(2, 8, 2, 256, None, None, None)
     with pytest.raises(native.MoeError) as ei:
         c.lookup(0, [0, 1, 2])
     assert ei.value.status == native.MOE_ERR_CAPACITY
     slots, miss = c.lookup(1, [5, 5, 5])
     assert len(set(slots)) == 1 and miss == [5]
     c.close()
-    r = native.SlotCache(1, 8, 8, 256, 0x1000, 0x2000, 0x3000)
+    r = native.SlotCache(1, 8, 8, 256, None, None, None)
     slots, miss = r.lookup(0, [3, 1])
     assert slots == [3, 1] and miss == [3, 1]          # first touch loads
+    r.fill(0, miss, side=0, compute=0)
     slots, miss = r.lookup(0, [3, 1, 7])
     assert slots == [3, 1, 7] and miss == [7]
-    assert r.stats() == {"hits": 0, "misses": 0, "h2d_bytes": 0}   # accounting bypassed
+    assert r.stats() == {"hits": 0, "misses": 0, "h2d_bytes": 2 * 256}   # accounting bypassed; first loads copied
     r.close()
 
 
 def test_slot_cache_injected_fill_failure_rolls_back(native):
-    c = native.SlotCache(1, 8, 4, 256, 0x1000, 0x2000, 0x3000)
+    c = native.SlotCache(1, 8, 4, 256, None, None, None)
     _, miss = c.lookup(0, [1, 2])
     c.inject_fill_failure(1)
     with pytest.raises(native.MoeError) as ei:
@@ -163,3 +129,25 @@ def test_slot_cache_injected_fill_failure_rolls_back(native):
     with pytest.raises(native.MoeError):
         c.fill(0, [5], side=0, compute=0)                 # never assigned by a lookup
     c.close()
+
+
+def test_slot_cache_lookup_without_fill_is_undone(native):
+    # a lookup whose misses were never copied must not leave them "resident":
+    # the next lookup misses them again rather than reading stale slot bytes
+    c = native.SlotCache(1, 8, 4, 256, None, None, None)
+    _, miss = c.lookup(0, [1, 2])
+    assert miss == [1, 2]
+    _, miss = c.lookup(0, [1, 2])                         # no fill in between
+    assert miss == [1, 2]
+    c.fill(0, miss, side=0, compute=0)
+    _, miss = c.lookup(0, [1, 2, 3])
+    assert miss == [3]
+    st = c.stats()
+    assert st["hits"] == 2 and st["h2d_bytes"] == 2 * 256   # the unfilled lookup copied nothing
+    c.close()
+
+
+def test_slot_cache_needs_all_memories_or_none(native):
+    with pytest.raises(native.MoeError) as ei:
+        native.SlotCache(1, 8, 4, 256, None, 0x2000, None)
+    assert ei.value.status == native.MOE_ERR_INVALID_ARG

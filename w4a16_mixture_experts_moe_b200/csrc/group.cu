@@ -237,8 +237,11 @@ extern "C" int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E, in
 // MOE_NOALLOC_MAX_PAIRS pairs and 256 experts, which every GPU that loads
 // this library keeps until the process exits. Host code must not use the
 // array's name as a device address (on the host it is only a stand-in), so
-// the address is looked up once per device with cudaGetSymbolAddress, with
-// that device current, on the first call made on it.
+// the address is looked up with cudaGetSymbolAddress with the device current.
+// A call made outside stream capture looks it up every time (a device reset
+// or a new primary context moves the array); a call made under capture
+// reuses the address of the last call on that device, so the first call on a
+// device belongs before any capture.
 namespace moe {
 
 constexpr size_t NOALLOC_SCRATCH_BYTES =
@@ -246,15 +249,17 @@ constexpr size_t NOALLOC_SCRATCH_BYTES =
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
-static int noalloc_scratch(void **out) {
+static int noalloc_scratch(cudaStream_t stream, void **out) {
   static std::mutex mu;
   static void *addr[64] = {nullptr};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_group_tokens_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= 64) return set_error(MOE_ERR_UNSUPPORTED, "moe_group_tokens_noalloc: device %d", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) cap = cudaStreamCaptureStatusActive;  // e.g. the legacy
+  std::lock_guard<std::mutex> lock(mu);                                                         // stream during a capture
+  if (!addr[dev] || cap == cudaStreamCaptureStatusNone) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p)
@@ -275,7 +280,7 @@ extern "C" int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, i
     return set_error(MOE_ERR_SHAPE, "moe_group_tokens_noalloc: T*k = %lld pairs exceeds the fixed scratch limit of %d",
                      (long long)(int64_t(T) * (k < 1 ? 1 : k)), MOE_NOALLOC_MAX_PAIRS);
   void *ws = nullptr;
-  const int st = noalloc_scratch(&ws);
+  const int st = noalloc_scratch(as_stream(stream), &ws);
   if (st != MOE_OK) return st;
   return moe_group_tokens(topk_ids, T, k, E, counts, offsets, sorted_pair, pair_pos, ws, NOALLOC_SCRATCH_BYTES,
                           stream);

@@ -37,6 +37,7 @@ struct moe_slot_cache {
   uint8_t *dev_slots;
   int32_t *dev_table;
   bool resident;
+  bool simulate;  // created without memory: policy and counters only
   // per layer
   std::vector<std::vector<int32_t>> owner;     // [layer][slot] expert or -1
   std::vector<std::vector<int32_t>> where;     // [layer][expert] slot or -1
@@ -59,14 +60,17 @@ extern "C" int slot_cache_create(moe_slot_cache **out, int layers, int E, int sl
   if (layers < 1 || E < 1 || E > MAX_E || slots < 1 || record_bytes < 256 || record_bytes % 256)
     return set_error(MOE_ERR_SHAPE, "slot_cache_create: layers=%d E=%d slots=%d record_bytes=%lld", layers, E, slots,
                      (long long)record_bytes);
-  if (!pinned_pool || !device_slots || !expert_slot)
-    return set_error(MOE_ERR_INVALID_ARG, "slot_cache_create: NULL pointer");
+  const bool simulate = !pinned_pool && !device_slots && !expert_slot;
+  if (!simulate && (!pinned_pool || !device_slots || !expert_slot))
+    return set_error(MOE_ERR_INVALID_ARG, "slot_cache_create: NULL pointer (pass all three memories, or none to "
+                     "simulate the policy)");
   moe_slot_cache *c = new moe_slot_cache();
   c->layers = layers; c->E = E; c->slots = slots; c->rec = record_bytes;
   c->pool = static_cast<const uint8_t *>(pinned_pool);
   c->dev_slots = static_cast<uint8_t *>(device_slots);
   c->dev_table = expert_slot;
   c->resident = slots >= E;
+  c->simulate = simulate;
   c->owner.assign(layers, std::vector<int32_t>(slots, -1));
   c->where.assign(layers, std::vector<int32_t>(E, -1));
   c->loaded.assign(layers, std::vector<uint8_t>(E, 0));
@@ -85,6 +89,22 @@ extern "C" int slot_cache_create(moe_slot_cache **out, int layers, int E, int sl
   return MOE_OK;
 }
 
+// Undoes the slot assignments of the layer's last lookup whose records were
+// never copied (a failed fill, or a lookup that no fill followed): those
+// experts and their slots go back to empty, so a later lookup misses them
+// again instead of reading a slot that holds stale bytes.
+static void rollback(moe_slot_cache *c, int layer) {
+  auto &ids = c->pending_ids[layer];
+  auto &sl = c->pending_slots[layer];
+  for (size_t i = 0; i < ids.size(); ++i) {
+    if (c->resident) { c->loaded[layer][ids[i]] = 0; continue; }
+    c->where[layer][ids[i]] = -1;
+    c->owner[layer][sl[i]] = -1;
+  }
+  ids.clear();
+  sl.clear();
+}
+
 extern "C" int slot_cache_lookup(moe_slot_cache *c, int layer, const int32_t *ids, int n, int32_t *slot_of_id,
                                  int32_t *miss_ids, int *n_miss) {
   using namespace moe;
@@ -98,8 +118,7 @@ extern "C" int slot_cache_lookup(moe_slot_cache *c, int layer, const int32_t *id
   auto &owner = c->owner[layer];
   auto &where = c->where[layer];
   auto &stamp = c->stamp[layer];
-  c->pending_ids[layer].clear();
-  c->pending_slots[layer].clear();
+  rollback(c, layer);  // the previous lookup's misses were never filled
   const uint64_t now = ++c->step[layer];
 
   // distinct ids, first occurrence order
@@ -159,18 +178,6 @@ static int ensure_events(moe_slot_cache *c, int layer) {
   return MOE_OK;
 }
 
-static void rollback(moe_slot_cache *c, int layer) {
-  auto &ids = c->pending_ids[layer];
-  auto &sl = c->pending_slots[layer];
-  for (size_t i = 0; i < ids.size(); ++i) {
-    if (c->resident) { c->loaded[layer][ids[i]] = 0; continue; }
-    c->where[layer][ids[i]] = -1;
-    c->owner[layer][sl[i]] = -1;
-  }
-  ids.clear();
-  sl.clear();
-}
-
 extern "C" int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss_ids, int n_miss, moe_stream_t side,
                                moe_stream_t compute) {
   using namespace moe;
@@ -186,6 +193,12 @@ extern "C" int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss
     --c->inject_fail;
     rollback(c, layer);
     return set_error(MOE_ERR_CUDA, "slot_cache_fill: injected fill failure (layer %d)", layer);
+  }
+  if (c->simulate) {  // no memory: the misses count as copied
+    c->h2d_bytes += uint64_t(n_miss) * uint64_t(c->rec);
+    c->pending_ids[layer].clear();
+    c->pending_slots[layer].clear();
+    return MOE_OK;
   }
   int st = ensure_events(c, layer);
   if (st != MOE_OK) { rollback(c, layer); return st; }
@@ -220,6 +233,7 @@ extern "C" int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss
 extern "C" int slot_cache_release(moe_slot_cache *c, int layer, moe_stream_t compute) {
   using namespace moe;
   if (!c || layer < 0 || layer >= c->layers) return set_error(MOE_ERR_INVALID_ARG, "slot_cache_release: bad argument");
+  if (c->simulate) return MOE_OK;
   int st = ensure_events(c, layer);
   if (st != MOE_OK) return st;
   cudaError_t e = cudaEventRecord(c->released[layer], as_stream(compute));
