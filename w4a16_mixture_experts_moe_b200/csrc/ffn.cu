@@ -25,8 +25,10 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, bool &bad) {
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-// x [T][H] BF16 -> FP16 copy, the decode path's gate/up input (exact for
-// BF16 values of magnitude <= 65504); flags values outside FP16's finite range.
+// x [T][H] BF16 -> FP16 copy, the decode path's gate/up input: exact for
+// BF16 values v with 2^-17 <= |v| <= 65504 and for zero; smaller magnitudes
+// round to a multiple of 2^-24 (absolute error at most 2^-25); values above
+// FP16's finite range are flagged.
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ x16,
                                                        int64_t n8, int32_t *err) {
   pdl_trigger();

@@ -25,8 +25,10 @@
 // Why FP16 operands: unpacking codes costs integer instructions, and FP16's
 // 10-bit mantissa lets a nibble sit at bits 4-7 of a half: one LOP3 yields
 // (1024 + u) and another (1024 + 16u) for the next code, with no shift. Codes
-// and BF16 activations are exact in FP16 (the activations while |x| <= 65504,
-// which the FP16 copy of x checks).
+// are exact in FP16. A BF16 value v is exact in FP16 when 2^-17 <= |v| <=
+// 65504 (or v = 0); a smaller one rounds to a multiple of 2^-24 (an absolute
+// error of at most 2^-25), and a larger one does not fit: the FP16 copy of x
+// and the h store flag MOE_DEVERR_RANGE for it.
 #include <cmath>
 
 #include "ffn.cuh"
@@ -216,6 +218,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
             for (int c = 0; c < 4; ++c) { ag[h][c] += red[q][sl][8 * h + c][lane]; au[h][c] += red[q][sl][8 * h + 4 + c][lane]; }
       }
     }
+    bool bad = false;  // an h outside FP16's finite range cannot be the down pass's operand
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int r = n0 + 2 * t + c;
@@ -223,11 +226,15 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
         uint16_t *hr = a.h + int64_t(lo + r) * a.I + row0 + g;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          hr[16 * h] = __half_as_ushort(__float2half_rn(bf16_to_f(f_to_bf16(silu_f(ag[h][c]) * au[h][c]))));
-          hr[16 * h + 8] = __half_as_ushort(__float2half_rn(bf16_to_f(f_to_bf16(silu_f(ag[h][2 + c]) * au[h][2 + c]))));
+          const float v0 = bf16_to_f(f_to_bf16(silu_f(ag[h][c]) * au[h][c]));
+          const float v1 = bf16_to_f(f_to_bf16(silu_f(ag[h][2 + c]) * au[h][2 + c]));
+          bad |= fabsf(v0) > 65504.f || fabsf(v1) > 65504.f;
+          hr[16 * h] = __half_as_ushort(__float2half_rn(v0));
+          hr[16 * h + 8] = __half_as_ushort(__float2half_rn(v1));
         }
       }
     }
+    if (bad) flag_error(a.err, MOE_DEVERR_RANGE);
   }
 }
 

@@ -36,15 +36,24 @@
 //   warp 18     one thread issues the TMA loads of the B ring (a 64 x 256
 //               FP16 box).
 // Why FP16 operands: q*s has at most 3 + 8 significant bits (|q| <= 8 and an
-// 8-bit BF16 scale significand) and FP16 holds 11, so the dequantised weight
-// is exact; a BF16 activation (8 significant bits) converts to FP16 exactly
-// too. The MMA then sums exact products in fp32, the same arithmetic as the
-// GEMV path (scale applied to fp32 group sums). This holds while activations
-// stay within FP16's range (|v| <= 65504; values below 2^-17 round by at most
-// 2^-25) and scales are >= 2^-14; a pre-pass converts x to FP16 and flags
-// MOE_DEVERR_RANGE for an activation out of range. The gate/up epilogue
-// rounds h to BF16 (the method's A16 intermediate) and stores that value in
-// FP16, which again is exact.
+// 8-bit BF16 scale significand) and is a multiple of the scale's last bit.
+// Each weight row is moved by a power of two 2^a (a per row, from its largest
+// scale: that scale times 2^a lies in [2^-4, 2^-3)), so the dequantised value
+// q*s*2^a has magnitude <= 1 and is exact in FP16 for every scale of the row
+// down to 2^-13 of the largest (a normal FP16 holds 11 significant bits; FP16
+// subnormals are multiples of 2^-24). The epilogue multiplies the row's fp32
+// sum by 2^-a, which is exact, so the tile computes x.(q*s) with exact
+// products summed in fp32, like the GEMV path (which applies each group scale
+// to an fp32 partial sum), whatever the weights' magnitude: without it a scale
+// below 2^-17 would be rounded and one above 8188 would overflow FP16. (The
+// target is deliberately small: rows moved up to |q*s*2^a| ~ 2^15 measured
+// far less accurate sums on the tensor cores, errors of up to 30 % at K =
+// 4096, while operands of magnitude <= 1 match the oracle.) A BF16 activation converts to FP16 exactly
+// when 2^-17 <= |v| <= 65504 (or v = 0); smaller ones round to a multiple of
+// 2^-24 (absolute error at most 2^-25). A pre-pass converts x to FP16 and
+// flags MOE_DEVERR_RANGE for an activation above 65504 in magnitude. The
+// gate/up epilogue rounds h to BF16 (the method's A16 intermediate), stores
+// that value in FP16 and flags the same error for an h that does not fit.
 // Both passes run two 128-row blocks of A against each activation box (gate
 // and up of the same features; or 256 consecutive down-output features), so
 // the two N = 256 accumulators fill all 512 tensor-memory columns with one
@@ -97,7 +106,7 @@ struct Cfg {
   static constexpr int ACC_COLS = NMAT * BN;          // columns per accumulator buffer
   static constexpr int TMEM_COLS = 512;
   static constexpr int NBUF = TMEM_COLS / ACC_COLS;   // accumulator buffers (1: two N = 256 blocks fill TMEM)
-  static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 4096 /*tables, barriers*/;
+  static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 6144 /*tables, barriers*/;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(S <= MAX_RING && CS <= MAX_RING, "ring depth");
   static_assert(B_OFF % 1024 == 0 && C_OFF % 1024 == 0, "swizzled buffers need 1024-byte alignment");
@@ -197,14 +206,23 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+// Two 32-lane x 16-column accumulator loads and the wait for them, in ONE asm
+// statement: the destination registers of tcgen05.ld hold their values only
+// after tcgen05.wait::ld, and a separate wait statement (tied to the loads
+// by nothing but a memory clobber) lets the compiler schedule arithmetic on
+// those registers ahead of it, reading whatever they held before.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, uint32_t (&a)[16], uint32_t (&b)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+        "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
+        "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+        "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ shared state
 struct Shared {
@@ -217,7 +235,12 @@ struct Shared {
   int32_t total_tiles;
   int32_t off[MAX_E + 1];    // group offsets
   int32_t tstart[MAX_E + 1]; // first tile of each expert
+  // power-of-two exponent of each weight row of a tile, written by the
+  // dequant warps at the tile's start, read by the epilogue after the tile's
+  // accumulator is complete; indexed by tile % ROWEXP_SLOTS ([block][row])
+  int16_t row_exp[4][2][128];
 };
+constexpr int ROWEXP_SLOTS = 4;  // tiles in flight between the two: at most three
 
 // Bounded wait: false (and the CTA-wide abort flag set) after WAIT_NS, or
 // as soon as another role aborted unless `drain` is set (a drain wait only
@@ -247,6 +270,25 @@ __device__ __noinline__ bool wait_bounded(Shared &sh, uint64_t *bar, uint32_t pa
 struct Tile {
   int e, lo, n0, nvalid, f0;
 };
+
+// v * 2^n for |n| <= 252, as two multiplications by exact powers of two
+// (each factor a normal fp32), so the result is exact unless it is subnormal.
+__device__ __forceinline__ float mul_pow2(float v, int n) {
+  const int n1 = n / 2, n2 = n - n1;
+  return v * __uint_as_float(uint32_t(127 + n1) << 23) * __uint_as_float(uint32_t(127 + n2) << 23);
+}
+
+// Exponent a of a weight row's power-of-two normalisation: the row's largest
+// BF16 scale times 2^a lies in [2^-4, 2^-3), so every dequantised weight
+// q*s*2^a has magnitude <= 1 (a = 0 for an all-zero row). Scales are never
+// negative, so their bit patterns order like their values.
+__device__ __forceinline__ int row_exponent(const uint16_t *srow, int G) {
+  uint32_t mx = 0;
+  for (int g = 0; g < G; ++g) mx = max(mx, uint32_t(srow[g]));
+  if (mx == 0) return 0;
+  const int e = min(127, max(-133, ilogbf(bf16_to_f(uint16_t(mx)))));  // floor(log2(largest scale))
+  return -4 - e;
+}
 
 template <int FW>
 __device__ __forceinline__ Tile decode_tile(const Shared &sh, int E, int FT, int t) {
@@ -319,7 +361,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (cnt > 0) {
           const int slot = a.expert_slot ? a.expert_slot[e] : e;
           if (slot >= 0 && slot < a.n_slots) v[i] = ((cnt + BN - 1) / BN) * FT;
-          else flag_error(a.err, MOE_DEVERR_NOT_RESIDENT);
+          else if (slot != MOE_SLOT_SKIP) flag_error(a.err, MOE_DEVERR_NOT_RESIDENT);
         }
       }
       local += v[i];
@@ -353,7 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Thread (p, i): weight row f0+i of the tile; p = the matrix (gate/up
     // pass) or the K half of the k-step (down pass).
     const int p = tid >> 7, i = tid & 127;
-    int deq_tile = -1, ks = 0;
+    int deq_tile = -1, ks = 0, deq_a = 0;
     const uint16_t *deq_srow = nullptr;
     const __half2 h1032 = __floats2half2_rn(1032.0f, 1032.0f);
     const __half2 h16th = __floats2half2_rn(0.0625f, 0.0625f);
@@ -372,6 +414,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         deq_srow = row < NOUT ? reinterpret_cast<const uint16_t *>(rec + (GATEUP ? (p ? a.off_us : a.off_gs) : a.off_ds)) +
                                     int64_t(row) * G
                               : nullptr;
+        deq_a = deq_srow ? row_exponent(deq_srow, G) : 0;
+        // the epilogue of this tile undoes the same power of two; the write is
+        // ordered before it by this tile's first a_full arrival, the MMAs and
+        // the tile's accumulator commit
+        sh.row_exp[deq_tile % ROWEXP_SLOTS][p][i] = int16_t(deq_a);
       }
       const uint16_t sbits = deq_srow ? deq_srow[(ks * BK) / GROUP] : uint16_t(0);  // one 32-byte line per row and tile
       const int cs = it % C::CS, as = it % C::S;
@@ -392,7 +439,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(&sh.c_free[cs]);  // the warp's codes are in registers: the slot may be refilled
       ok = __all_sync(0xffffffffu, wait_bounded(sh, &sh.s_free[as], ((it / C::S) & 1) ^ 1, a.err));
       if (!ok) break;
-      const __half2 sc = __half2half2(__float2half_rn(bf16_to_f(sbits)));
+      const __half2 sc = __half2half2(__float2half_rn(mul_pow2(bf16_to_f(sbits), deq_a)));  // s * 2^a, exact
       constexpr int NW = 8;
       const int c0 = 0;
       uint8_t *arow = ringA + as * C::A_BYTES + p * (BM * BK * 2) + i * 128;
@@ -429,40 +476,47 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
       const Tile tl = decode_tile<C::FW>(sh, E, FT, t);
       const int b = tl_i % C::NBUF;
+      const int f = tl.f0 + frow;
       if (!__all_sync(0xffffffffu, wait_bounded(sh, &sh.tmem_full[b], (tl_i / C::NBUF) & 1, a.err))) break;
       tc_fence_after();
+      // undo the dequant warps' power-of-two row normalisation: block 0 =
+      // gate row f (gate/up pass) or down row f; block 1 = up row f or down
+      // row f + 128. (The epilogue issues no global loads of its own ahead of
+      // the accumulator wait: a version that read the row scales there, as
+      // the dequant warps do, measured corrupted tiles that no barrier
+      // analysis explained, while the same loads in the dequant warps and
+      // plain delays in the epilogue did not.)
+      const float unscale0 = mul_pow2(1.0f, -int(sh.row_exp[tl_i % ROWEXP_SLOTS][0][frow]));
+      const float unscale1 = mul_pow2(1.0f, -int(sh.row_exp[tl_i % ROWEXP_SLOTS][1][frow]));
       const uint32_t tbase = tmem + (uint32_t(q * 32) << 16) + b * C::ACC_COLS;
-      const int f = tl.f0 + frow;
       const int j_lo = half * (BN / 2), j_hi = min(tl.nvalid, j_lo + BN / 2);
       const int64_t row0 = int64_t(tl.lo + tl.n0);
       for (int j0 = j_lo; j0 < j_hi; j0 += 16) {
-        uint32_t g[16];
-        tmem_ld16(tbase + j0, g);
+        uint32_t g[16], u[16];  // gate/up: gate and up sums; down: the two 128-row output blocks
+        tmem_ld16x2(tbase + j0, tbase + BN + j0, g, u);
         if (GATEUP) {
-          uint32_t u[16];
-          tmem_ld16(tbase + BN + j0, u);
-          tmem_wait_ld();
           uint16_t *hp = a.h + (row0 + j0) * NOUT + f;
+          bool bad = false;  // an h outside FP16's finite range cannot be the down pass's operand
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             if (j0 + jj < j_hi) {
-              const float gv = __uint_as_float(g[jj]), uv = __uint_as_float(u[jj]);
+              const float gv = __uint_as_float(g[jj]) * unscale0, uv = __uint_as_float(u[jj]) * unscale1;
               const float hv = bf16_to_f(f_to_bf16(silu_f(gv) * uv));  // A16: h is BF16
+              bad |= fabsf(hv) > 65504.f;
               hp[jj * NOUT] = __half_as_ushort(__float2half_rn(hv));
             }
           }
+          if (bad) flag_error(a.err, MOE_DEVERR_RANGE);
         } else {
-          uint32_t g2[16];
-          tmem_ld16(tbase + BN + j0, g2);  // second 128-row block
-          tmem_wait_ld();
+          const uint32_t (&g2)[16] = u;  // second 128-row block
           float *yp = a.y + (row0 + j0) * NOUT + f;
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj)
-            if (j0 + jj < j_hi) yp[jj * NOUT] = __uint_as_float(g[jj]);
+            if (j0 + jj < j_hi) yp[jj * NOUT] = __uint_as_float(g[jj]) * unscale0;
           if (f + BM < NOUT) {
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj)
-              if (j0 + jj < j_hi) yp[jj * NOUT + BM] = __uint_as_float(g2[jj]);
+              if (j0 + jj < j_hi) yp[jj * NOUT + BM] = __uint_as_float(g2[jj]) * unscale1;
           }
         }
       }
