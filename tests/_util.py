@@ -29,3 +29,18 @@ def torch_weights_source(gate, up, down):
     def weights_of(e):
         return gate[e].double().numpy(), up[e].double().numpy(), down[e].double().numpy()
     return weights_of
+
+
+def assert_logits_close(got, ref, x, wr, what=""):
+    """Router logits: one BF16 rounding of an fp32 sum taken in any order is
+    within one BF16 ulp of the fp64 oracle's rounded sum plus the fp32
+    summation bound (H - 1) 2^-24 sum_h |x w| (which matters near zero,
+    where a BF16 ulp is tiny and the fp32 sum cancels)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    wr = np.asarray(wr, dtype=np.float64)
+    ulp = np.ldexp(1.0, np.frexp(ref)[1] - 8)
+    bound = ulp + (x.shape[1] - 1) * 2.0 ** -24 * (np.abs(x) @ np.abs(wr).T)
+    bad = ~(np.abs(got - ref) <= bound)
+    assert not bad.any(), f"{what}: {int(bad.sum())} logits beyond one BF16 ulp + the fp32 summation bound"
