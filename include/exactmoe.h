@@ -75,8 +75,9 @@ enum {
   MOE_DEVERR_EXPERT_ID = 1,   /* a top-k id outside [0, E) */
   MOE_DEVERR_NOT_RESIDENT = 2,/* an active expert has no valid slot */
   MOE_DEVERR_TIMEOUT = 3,     /* a bounded pipeline wait ran out */
-  MOE_DEVERR_RANGE = 4        /* an activation outside FP16 range on the
-                                 tensor-core path (|x| > 65504) */
+  MOE_DEVERR_RANGE = 4        /* an activation x or an expert intermediate h
+                                 outside FP16's finite range (|v| > 65504):
+                                 the FFN's FP16 operand copies cannot hold it */
 };
 
 /* Message for the last failed call on this host thread ("" if none). */
@@ -177,19 +178,26 @@ int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E,
  * every GPU that loads the library holds until the process exits; it allows
  * at most MOE_NOALLOC_MAX_PAIRS = T*k pairs (larger calls return
  * MOE_ERR_SHAPE and launch nothing). This call allocates nothing and calls no
- * cudaMalloc/cudaFree. The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture. All calls share the one array: calls whose
- * kernels overlap on the GPU (other streams, other host threads) race and
- * corrupt each other's results, so serialise them. Device-side errors are not
- * reported through a workspace word here: a pair with an out-of-range id gets
- * pair_pos = -1, which the caller can check.
+ * cudaMalloc/cudaFree. It looks up the array's device address
+ * (cudaGetSymbolAddress) with the current device on every call made outside
+ * stream capture, so a device reset does not leave it stale; a call under
+ * capture reuses the address found by the last call on that device, so make
+ * the first call on a device before any stream capture. All calls share the
+ * one array: calls whose kernels overlap on the GPU (other streams, other
+ * host threads) race and corrupt each other's results, so serialise them.
+ * Device-side errors are not reported through a workspace word here (the
+ * array's error word is written but never read): a pair with an out-of-range
+ * id gets pair_pos = -1, which the caller can check.
  */
 #define MOE_NOALLOC_MAX_PAIRS 65536
 int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E,
                              int32_t *counts, int32_t *offsets,
                              int32_t *sorted_pair, int32_t *pair_pos,
                              moe_stream_t stream);
+
+/* expert_slot value of an expert that a grouped FFN call leaves to another
+ * call (another wave of the same step). */
+#define MOE_SLOT_SKIP (-2)
 
 /* FFN execution paths. */
 #define MOE_PATH_AUTO 0 /* chosen from the average rows per expert, T*k/E */
@@ -209,20 +217,29 @@ int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E,
  *                (moe_expert_record_layout(H, I).bytes or larger, multiple
  *                of 256).
  *   expert_slot  [E] int32 record index of each expert in the bank, or NULL
- *                for the identity (record e holds expert e). An active
- *                expert whose slot is outside [0, n_slots) is skipped and
- *                flagged (MOE_DEVERR_NOT_RESIDENT).
+ *                for the identity (record e holds expert e). An expert marked
+ *                MOE_SLOT_SKIP is not computed by this call (its rows of y
+ *                are left as they are: another call of the same step, one
+ *                wave of a slot cache, computes them). An active expert with
+ *                any other slot outside [0, n_slots) is skipped and flagged
+ *                (MOE_DEVERR_NOT_RESIDENT).
  *   y            [T*k][H] fp32, rows in sorted order (the expert outputs
  *                are kept unrounded until the combine).
  *   ws           at least moe_ffn_workspace_size(T, k, E, H, I, path) bytes,
  *                256-byte aligned, zeroed once before first use; holds the
  *                error word, h and (tensor-core path) an FP16 copy of x.
- * Both paths form exact products x*(q*s) and sum them in fp32, on FP16 copies
- * of the activations (exact for BF16 values up to 65504 in magnitude; larger
- * ones are flagged MOE_DEVERR_RANGE): the GEMV path multiplies FP16 codes q
- * and applies each group's scale to the fp32 partial sum over that group; the
- * tensor-core path dequantises q*s to FP16 (exact: at most 11 significant
- * bits).
+ * Both paths sum products of the weights q*s and FP16 copies of the
+ * activations (x, and h for the down pass) in fp32. A BF16 value v copies to
+ * FP16 exactly when 2^-17 <= |v| <= 65504 or v = 0; a smaller magnitude
+ * rounds to a multiple of 2^-24 (absolute error <= 2^-25), and a larger one
+ * is flagged MOE_DEVERR_RANGE (for h as well as x; the affected rows are then
+ * not meaningful). The GEMV path multiplies FP16 codes q and applies each
+ * group's scale to the fp32 partial sum over that group, exact for every
+ * scale. The tensor-core path dequantises q*s*2^a to FP16, with a per-row
+ * power of two 2^a that brings the row's largest scale to [2^-4, 2^-3) and is
+ * undone exactly on the fp32 sum: exact for every group whose scale is at
+ * least 2^-13 of its row's largest (smaller ones are rounded to a multiple of
+ * 2^-24 relative to that normalisation).
  */
 size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path);
 int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair,
@@ -271,8 +288,22 @@ int moe_read_device_error(void *ws, moe_stream_t stream, int32_t *code);
  * events per layer; all memory is the caller's:
  *   pinned_pool   host, page-locked, [layers][E] records of record_bytes.
  *   device_slots  device, [layers][slots] records of record_bytes.
- *   expert_slot   device, [layers][E] int32, the table the FFN reads
- *                 (-1 = not resident). slot_cache_fill keeps it current.
+ *   expert_slot   device, [layers][E] int32, the table the FFN reads.
+ *                 slot_cache_fill writes it for the layer's last lookup: the
+ *                 looked-up experts' slots; MOE_SLOT_SKIP for the other
+ *                 experts of a step planned by slot_cache_plan_waves; -1 for
+ *                 every other expert (flagged by the FFN if a token selects
+ *                 it). Initialise it to -1.
+ * With all three NULL the cache only simulates the policy (no CUDA call is
+ * made): slot_cache_fill counts the misses' bytes as copied and copies
+ * nothing, slot_cache_release does nothing. Hit rates and traffic of a
+ * routing trace can be measured that way without a GPU.
+ *
+ * Replacement policy (the pages name none; this is the library's reading):
+ * a step's distinct ids are taken in first-occurrence order; ids already held
+ * are hits and their slots are protected for the step; each miss takes the
+ * lowest empty slot, else the least recently used unprotected slot, the lower
+ * slot index on ties.
  */
 typedef struct moe_slot_cache moe_slot_cache;
 
@@ -285,21 +316,41 @@ int slot_cache_create(moe_slot_cache **out, int layers, int E, int slots,
  * the least recently used slot that this step does not need, and listed in
  * miss_ids (host, capacity n). Duplicate ids count once. More distinct ids
  * than slots -> MOE_ERR_CAPACITY. Resident caches (slots >= E) never miss
- * and count nothing. */
+ * and count nothing. If the layer's previous lookup assigned slots that no
+ * successful slot_cache_fill copied, those assignments are undone first
+ * (the experts count as absent again). */
 int slot_cache_lookup(moe_slot_cache *c, int layer, const int32_t *ids_host,
                       int n, int32_t *slot_of_id_host,
                       int32_t *miss_ids_host, int *n_miss);
 
 /* Copies the records of the missed experts from the pinned pool into their
  * slots on `side` (one cudaMemcpyAsync each, after the layer's previous
- * readers released it), updates the layer's device expert_slot table, and
- * makes `compute` wait for all of it. */
+ * readers released it), makes `compute` wait for the copies, and rewrites the
+ * layer's device expert_slot table on `compute` when it changes (a one-block
+ * kernel). Call it after every lookup, also with n_miss = 0. */
 int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss_ids_host,
                     int n_miss, moe_stream_t side, moe_stream_t compute);
 
 /* Marks the end of this step's reads of `layer`'s slots on `compute`; the
  * next fill of the layer waits for this point before overwriting a slot. */
 int slot_cache_release(moe_slot_cache *c, int layer, moe_stream_t compute);
+
+/*
+ * Cache-sized fused waves (Figure 1 caption: the active experts execute in
+ * cache-sized fused waves). Splits the n expert ids (host) one step of
+ * `layer` needs into waves of at most `slots` distinct experts: the
+ * distinct ids in first-occurrence order, those already held in a slot
+ * first (so they run before anything can evict them), cut into consecutive
+ * waves. Writes the ordered ids to wave_ids (host, capacity n), the start of
+ * wave w to wave_start[w] (host, capacity n + 1; wave_start[n_waves] is the
+ * total) and the count to *n_waves (0 when n == 0). Per wave: lookup of its
+ * ids, fill, one grouped FFN call with the same grouping of the whole step
+ * (it computes only that wave's experts), release; the combine follows the
+ * last wave. Planning marks the step's experts so that each wave's table
+ * skips the others; call it at the start of every step run in waves.
+ */
+int slot_cache_plan_waves(moe_slot_cache *c, int layer, const int32_t *ids_host, int n,
+                          int32_t *wave_ids_host, int32_t *wave_start_host, int *n_waves);
 
 int slot_cache_stats(const moe_slot_cache *c, uint64_t *hits,
                      uint64_t *misses, uint64_t *h2d_bytes);

@@ -477,6 +477,19 @@ class SlotCacheLRU:
             loaded.append(v)
         return [self.slot_of(v) for v in ids], loaded, evicted
 
+    def plan_waves(self, ids):
+        """Cache-sized waves (Figure 1 caption: active experts execute in
+        cache-sized fused waves): the step's distinct ids in first-occurrence
+        order, those already held in a slot first, cut into consecutive
+        waves of at most S ids. Each wave is then one lookup."""
+        distinct = []
+        for v in (int(i) for i in ids):
+            if v not in distinct:
+                distinct.append(v)
+        held = [v for v in distinct if self.slot_of(v) is not None]
+        order = held + [v for v in distinct if v not in held]
+        return [order[i:i + self.S] for i in range(0, len(order), self.S)]
+
     def h2d_bytes(self, record_bytes: int) -> int:
         """Host-to-device bytes moved so far: one record per load."""
         return self.loads * int(record_bytes)

@@ -13,8 +13,8 @@ E=64 experts, top-8):
   seed 10000 + (l*E + e)*3 + m;
 * skewed routing: a per-expert logit offset log(Zipf(s=1.2)) where the
   expert's index is its rank;
-* slot-cache decode routing: per layer, drawn so that each expert of the
-  previous step is kept with probability 0.5.
+* slot-cache decode routing: per layer and token stream, drawn so that each
+  expert of the previous step is kept with probability 0.5.
 
 Every tensor has its own seed, so a test can regenerate any single expert
 without generating the rest. On the CPU the values come from torch's seeded
@@ -84,15 +84,17 @@ def zipf_log_bias(E: int, s: float = 1.2) -> np.ndarray:
 
 
 def drawn_routing(layer: int, E: int, k: int, steps: int,
-                  keep_p: float = 0.5) -> np.ndarray:
+                  keep_p: float = 0.5, stream: int = 0) -> np.ndarray:
     """Expert ids [steps][k] for decode at one token per step.
 
     Step 0 picks k distinct experts uniformly. Each later step keeps every
     expert of the previous step independently with probability keep_p, then
     fills the remaining places uniformly (without replacement) from the experts
-    the previous step did not use. Ids within a step are ascending.
+    the previous step did not use. Ids within a step are ascending. Decode at
+    T tokens per step draws T independent streams (stream = 0 .. T-1, seed
+    500 + layer + 1000 * stream; stream 0 is the one-token recipe).
     """
-    rng = np.random.Generator(np.random.PCG64(DRAWN_ROUTING_SEED + layer))
+    rng = np.random.Generator(np.random.PCG64(DRAWN_ROUTING_SEED + layer + 1000 * stream))
     out = np.empty((steps, k), dtype=np.int32)
     prev = np.sort(rng.choice(E, size=k, replace=False))
     out[0] = prev

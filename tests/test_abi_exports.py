@@ -7,6 +7,7 @@ import glob
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -151,3 +152,30 @@ def test_slot_cache_needs_all_memories_or_none(native):
     with pytest.raises(native.MoeError) as ei:
         native.SlotCache(1, 8, 4, 256, None, 0x2000, None)
     assert ei.value.status == native.MOE_ERR_INVALID_ARG
+
+
+def test_slot_cache_waves_match_oracle(native):
+    """Steps needing more experts than slots run in waves: the library's plan
+    and each wave's lookup match the oracle's policy (simulation mode)."""
+    import synth
+    from oracle import exactmoe_oracle as o
+    E, S, k, T, steps = 64, 16, 8, 4, 60
+    c = native.SlotCache(1, E, S, 256, None, None, None)
+    model = o.SlotCacheLRU(E, S)
+    rng = np.random.default_rng(17)
+    waves_seen = 0
+    for s in range(steps):
+        ids = [int(v) for v in rng.integers(0, E, size=T * k)] if s % 3 else \
+              [int(v) for v in synth.drawn_routing(0, E, k, steps)[s]]
+        waves = c.plan_waves(0, ids)
+        assert waves == model.plan_waves(ids), s
+        waves_seen += len(waves)
+        for w in waves:
+            got = c.lookup(0, w)
+            slots, loaded, _ = model.lookup(w)
+            assert got == (slots, loaded), s
+            c.fill(0, got[1], side=0, compute=0)
+    st = c.stats()
+    assert (st["hits"], st["misses"], st["h2d_bytes"]) == (model.hits, model.misses, model.h2d_bytes(256))
+    assert waves_seen > steps                       # some steps needed more than one wave
+    c.close()

@@ -342,6 +342,35 @@ def test_slot_cache_hand_worked_trace():
     assert c.h2d_bytes(1000) == 1000 * r["loads"]
 
 
+def test_slot_cache_waves_hand_worked():
+    g = json.load(open(LRU_GOLDEN))["waves"]
+    c = o.SlotCacheLRU(g["E"], g["slots"])
+    for st in g["steps"]:
+        waves = c.plan_waves(st["ids"])
+        assert waves == st["waves"], st
+        for w, want in zip(waves, st["per_wave"]):
+            slots, loaded, evicted = c.lookup(w)
+            assert (slots, loaded, evicted) == (want["slot_of_ids"], want["loaded"], want["evicted"]), st
+        assert (c.hits, c.misses) == (st["hits"], st["misses"]), st
+
+
+def test_slot_cache_waves_cover_each_expert_once():
+    # the waves of a step are a partition of its distinct ids, none larger
+    # than the cache, held ids first; with S >= distinct there is one wave
+    rng = np.random.default_rng(8)
+    c = o.SlotCacheLRU(20, 4)
+    for _ in range(100):
+        ids = [int(v) for v in rng.integers(0, 20, size=rng.integers(1, 13))]
+        held = {v for v in ids if c.slot_of(v) is not None}
+        waves = c.plan_waves(ids)
+        flat = [v for w in waves for v in w]
+        assert sorted(flat) == sorted(set(ids)) and all(1 <= len(w) <= 4 for w in waves)
+        assert set(flat[:len(held)]) == held
+        for w in waves:
+            c.lookup(w)
+    assert o.SlotCacheLRU(20, 16).plan_waves([3, 1, 3, 7]) == [[3, 1, 7]]
+
+
 @pytest.mark.parametrize("S", [1, 2, 3, 5, 8])
 def test_slot_cache_one_id_per_step_equals_library_lru(S):
     # with one expert per step the policy is a plain LRU cache of S entries:

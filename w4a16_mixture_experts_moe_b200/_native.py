@@ -25,6 +25,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_CUDA, MOE_ERR_CAPACITY, MOE_
 MOE_DEVERR_NONE, MOE_DEVERR_EXPERT_ID, MOE_DEVERR_NOT_RESIDENT, MOE_DEVERR_TIMEOUT, MOE_DEVERR_RANGE = range(5)
 MOE_RENORM, MOE_LOGITS_GIVEN, MOE_IDS_GIVEN = 1, 2, 4
 MOE_PATH_AUTO, MOE_PATH_GEMV, MOE_PATH_TC = 0, 1, 2
+MOE_SLOT_SKIP = -2
 
 _p = C.c_void_p
 _i = C.c_int
@@ -57,6 +58,7 @@ SIGNATURES = {
     "slot_cache_lookup": (_i, [_p, _i, _p, _i, _p, _p, C.POINTER(_i)]),
     "slot_cache_fill": (_i, [_p, _i, _p, _i, _p, _p]),
     "slot_cache_release": (_i, [_p, _i, _p]),
+    "slot_cache_plan_waves": (_i, [_p, _i, _p, _i, _p, _p, C.POINTER(_i)]),
     "slot_cache_stats": (_i, [_p, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]),
     "slot_cache_inject_fill_failure": (_i, [_p, _i]),
     "slot_cache_destroy": (None, [_p]),
@@ -203,6 +205,16 @@ class SlotCache:
 
     def release(self, layer, compute=None):
         _check(lib.slot_cache_release(self.h, layer, _stream(compute)))
+
+    def plan_waves(self, layer, ids):
+        """ids: sequence of ints. Returns the waves as lists of distinct ids."""
+        n = len(ids)
+        arr = (C.c_int32 * max(n, 1))(*ids)
+        wid = (C.c_int32 * max(n, 1))()
+        wst = (C.c_int32 * (n + 1))()
+        nw = C.c_int(0)
+        _check(lib.slot_cache_plan_waves(self.h, layer, _addr(arr), n, _addr(wid), _addr(wst), C.byref(nw)))
+        return [list(wid[wst[w]:wst[w + 1]]) for w in range(nw.value)]
 
     def stats(self):
         h, m, b = C.c_uint64(), C.c_uint64(), C.c_uint64()

@@ -31,11 +31,13 @@ struct FfnArgs {
 // calls still to be launched with their producers stalled.
 int take_tc_stall();
 
-// Record of expert e, or nullptr (and the error flagged) if it has no slot.
+// Record of expert e, or nullptr if this call does not compute it: an expert
+// marked MOE_SLOT_SKIP (another wave's) silently, any other slot outside
+// [0, n_slots) with the error flagged.
 __device__ __forceinline__ const uint8_t *expert_record(const FfnArgs &a, int e) {
   const int slot = a.expert_slot ? a.expert_slot[e] : e;
   if (slot < 0 || slot >= a.n_slots) {
-    flag_error(a.err, MOE_DEVERR_NOT_RESIDENT);
+    if (slot != MOE_SLOT_SKIP) flag_error(a.err, MOE_DEVERR_NOT_RESIDENT);
     return nullptr;
   }
   return a.bank + int64_t(slot) * a.rec;

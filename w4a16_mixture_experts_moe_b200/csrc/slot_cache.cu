@@ -9,11 +9,18 @@
 // least recently used slot that the current step does not need and is filled
 // with one cudaMemcpyAsync of the expert's whole record (packed codes and
 // scales, no dequantised copy) on a side stream. The layer's device table
-// expert -> slot is rewritten by a one-block kernel whose argument carries the
-// whole table, so no host buffer has to outlive the call.
+// expert -> slot names exactly the experts of the last lookup; when a step
+// needs more experts than there are slots (Figure 1 caption: active experts
+// run in cache-sized fused waves), slot_cache_plan_waves splits it, and the
+// step's experts outside the current wave are marked MOE_SLOT_SKIP, so each
+// wave's grouped FFN call computes that wave's experts and no other. The table
+// is rewritten by a one-block kernel on the compute stream, after the
+// previous reader of the table, whose argument carries the whole table, so no
+// host buffer has to outlive the call.
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <vector>
 
 #include "common.cuh"
@@ -48,6 +55,9 @@ struct moe_slot_cache {
   std::vector<bool> release_recorded;
   // misses of the last lookup per layer, for rollback if the fill fails
   std::vector<std::vector<int32_t>> pending_ids, pending_slots;
+  std::vector<std::vector<int32_t>> step_ids;    // [layer] distinct ids of the last lookup
+  std::vector<std::vector<uint8_t>> planned;     // [layer][expert] in the step last planned in waves
+  std::vector<std::vector<int32_t>> table_host;  // [layer] the device table as last written (empty: unknown)
   uint64_t hits = 0, misses = 0, h2d_bytes = 0;
   int inject_fail = 0;
 };
@@ -81,6 +91,9 @@ extern "C" int slot_cache_create(moe_slot_cache **out, int layers, int E, int sl
   c->release_recorded.assign(layers, false);
   c->pending_ids.assign(layers, {});
   c->pending_slots.assign(layers, {});
+  c->step_ids.assign(layers, {});
+  c->planned.assign(layers, std::vector<uint8_t>(E, 0));
+  c->table_host.assign(layers, {});
   if (c->resident) {
     for (int l = 0; l < layers; ++l)
       for (int e = 0; e < E; ++e) { c->owner[l][e] = e; c->where[l][e] = e; }
@@ -127,7 +140,11 @@ extern "C" int slot_cache_lookup(moe_slot_cache *c, int layer, const int32_t *id
   for (int i = 0; i < n; ++i)
     if (!seen[ids[i]]) { seen[ids[i]] = 1; uniq.push_back(ids[i]); }
   if (int(uniq.size()) > c->slots)
-    return set_error(MOE_ERR_CAPACITY, "slot_cache_lookup: %d distinct experts > %d slots", int(uniq.size()), c->slots);
+    return set_error(MOE_ERR_CAPACITY, "slot_cache_lookup: %d distinct experts > %d slots (plan waves with "
+                     "slot_cache_plan_waves)", int(uniq.size()), c->slots);
+  c->step_ids[layer] = uniq;
+  for (int32_t e : uniq)  // a lookup outside the planned step ends that plan
+    if (!c->planned[layer][e]) { std::fill(c->planned[layer].begin(), c->planned[layer].end(), 0); break; }
 
   if (c->resident) {  // every expert owns its slot; only first touches load
     for (int32_t e : uniq)
@@ -184,49 +201,102 @@ extern "C" int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss
   if (!c || (n_miss > 0 && !miss_ids)) return set_error(MOE_ERR_INVALID_ARG, "slot_cache_fill: NULL pointer");
   if (layer < 0 || layer >= c->layers || n_miss < 0)
     return set_error(MOE_ERR_INVALID_ARG, "slot_cache_fill: layer=%d n_miss=%d", layer, n_miss);
-  if (n_miss == 0) return MOE_OK;
   for (int i = 0; i < n_miss; ++i)
     if (miss_ids[i] < 0 || miss_ids[i] >= c->E || c->where[layer][miss_ids[i]] < 0)
       return set_error(MOE_ERR_INVALID_ARG, "slot_cache_fill: id %d was not assigned a slot by slot_cache_lookup",
                        miss_ids[i]);
-  if (c->inject_fail > 0) {
+  if (n_miss > 0 && c->inject_fail > 0) {
     --c->inject_fail;
     rollback(c, layer);
     return set_error(MOE_ERR_CUDA, "slot_cache_fill: injected fill failure (layer %d)", layer);
   }
+  // the table the FFN reads: the last lookup's experts in their slots, the
+  // other experts of a step planned in waves skipped, every other expert
+  // absent (-1: flagged if a token selects it)
+  std::vector<int32_t> table(c->E, -1);
+  for (int x = 0; x < c->E; ++x)
+    if (c->planned[layer][x]) table[x] = MOE_SLOT_SKIP;
+  for (int32_t x : c->step_ids[layer]) table[x] = c->where[layer][x];
+  const bool table_changed = table != c->table_host[layer];
   if (c->simulate) {  // no memory: the misses count as copied
     c->h2d_bytes += uint64_t(n_miss) * uint64_t(c->rec);
     c->pending_ids[layer].clear();
     c->pending_slots[layer].clear();
+    c->table_host[layer] = table;
     return MOE_OK;
   }
-  int st = ensure_events(c, layer);
-  if (st != MOE_OK) { rollback(c, layer); return st; }
+  if (n_miss == 0 && !table_changed) return MOE_OK;
   cudaStream_t s = as_stream(side), cs = as_stream(compute);
   cudaError_t e = cudaSuccess;
-  if (c->release_recorded[layer]) e = cudaStreamWaitEvent(s, c->released[layer], 0);
-  for (int i = 0; i < n_miss && e == cudaSuccess; ++i) {
-    const int id = miss_ids[i];
-    const int slot = c->where[layer][id];
-    uint8_t *dst = c->dev_slots + (int64_t(layer) * c->slots + slot) * c->rec;
-    const uint8_t *src = c->pool + (int64_t(layer) * c->E + id) * c->rec;
-    e = cudaMemcpyAsync(dst, src, size_t(c->rec), cudaMemcpyHostToDevice, s);
+  if (n_miss > 0) {
+    int st = ensure_events(c, layer);
+    if (st != MOE_OK) { rollback(c, layer); return st; }
+    if (c->release_recorded[layer]) e = cudaStreamWaitEvent(s, c->released[layer], 0);
+    for (int i = 0; i < n_miss && e == cudaSuccess; ++i) {
+      const int id = miss_ids[i];
+      const int slot = c->where[layer][id];
+      uint8_t *dst = c->dev_slots + (int64_t(layer) * c->slots + slot) * c->rec;
+      const uint8_t *src = c->pool + (int64_t(layer) * c->E + id) * c->rec;
+      e = cudaMemcpyAsync(dst, src, size_t(c->rec), cudaMemcpyHostToDevice, s);
+    }
+    if (e != cudaSuccess) {
+      rollback(c, layer);
+      return set_error(MOE_ERR_CUDA, "slot_cache_fill: copy: %s", cudaGetErrorString(e));
+    }
+    e = cudaEventRecord(c->filled[layer], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, c->filled[layer], 0);
+    if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "slot_cache_fill: %s", cudaGetErrorString(e));
+    c->h2d_bytes += uint64_t(n_miss) * uint64_t(c->rec);
   }
-  if (e != cudaSuccess) {
-    rollback(c, layer);
-    return set_error(MOE_ERR_CUDA, "slot_cache_fill: copy: %s", cudaGetErrorString(e));
-  }
-  SlotTable table;
-  for (int x = 0; x < c->E; ++x) table.slot_of[x] = c->where[layer][x];
-  write_slot_table_kernel<<<1, 256, 0, s>>>(c->dev_table + int64_t(layer) * c->E, c->E, table);
-  count_launches(1);
-  e = cudaGetLastError();
-  if (e == cudaSuccess) e = cudaEventRecord(c->filled[layer], s);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, c->filled[layer], 0);
-  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "slot_cache_fill: %s", cudaGetErrorString(e));
-  c->h2d_bytes += uint64_t(n_miss) * uint64_t(c->rec);
   c->pending_ids[layer].clear();
   c->pending_slots[layer].clear();
+  if (table_changed) {
+    SlotTable t;
+    for (int x = 0; x < c->E; ++x) t.slot_of[x] = table[x];
+    write_slot_table_kernel<<<1, 256, 0, cs>>>(c->dev_table + int64_t(layer) * c->E, c->E, t);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      c->table_host[layer].clear();
+      return set_error(MOE_ERR_CUDA, "slot_cache_fill: table: %s", cudaGetErrorString(e));
+    }
+    count_launches(1);
+    c->table_host[layer] = table;
+  }
+  return MOE_OK;
+}
+
+extern "C" int slot_cache_plan_waves(moe_slot_cache *c, int layer, const int32_t *ids, int n,
+                                     int32_t *wave_ids, int32_t *wave_start, int *n_waves) {
+  using namespace moe;
+  if (!c || !n_waves || (n > 0 && (!ids || !wave_ids || !wave_start)))
+    return set_error(MOE_ERR_INVALID_ARG, "slot_cache_plan_waves: NULL pointer");
+  if (layer < 0 || layer >= c->layers || n < 0)
+    return set_error(MOE_ERR_INVALID_ARG, "slot_cache_plan_waves: layer=%d n=%d", layer, n);
+  for (int i = 0; i < n; ++i)
+    if (ids[i] < 0 || ids[i] >= c->E)
+      return set_error(MOE_ERR_INVALID_ARG, "slot_cache_plan_waves: id %d out of range", ids[i]);
+  *n_waves = 0;
+  if (n == 0) return MOE_OK;
+  // distinct ids, first occurrence order; those whose records are in a slot
+  // (copied by a completed fill) come first, so they run before any eviction
+  std::vector<uint8_t> seen(c->E, 0), pending(c->E, 0);
+  for (int32_t x : c->pending_ids[layer]) pending[x] = 1;
+  std::vector<int32_t> held, absent;
+  for (int i = 0; i < n; ++i) {
+    const int x = ids[i];
+    if (seen[x]) continue;
+    seen[x] = 1;
+    const bool in_slot = c->resident ? c->loaded[layer][x] != 0 : c->where[layer][x] >= 0;
+    (in_slot && !pending[x] ? held : absent).push_back(x);
+  }
+  int m = 0;
+  for (int32_t x : held) wave_ids[m++] = x;
+  for (int32_t x : absent) wave_ids[m++] = x;
+  for (int x = 0; x < c->E; ++x) c->planned[layer][x] = seen[x];
+  int w = 0;
+  for (int start = 0; start < m; start += c->slots) wave_start[w++] = start;
+  wave_start[w] = m;
+  *n_waves = w;
   return MOE_OK;
 }
 
