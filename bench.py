@@ -40,13 +40,14 @@ SWEEP_T = (1, 4, 16, 64)
 METRIC = "MoE-layer tokens/s; HBM GB/s (decode) and TC TFLOP/s (prefill) vs B200 peak"
 SHAPES = {"olmoe": (2048, 1024, 64, 8), "wide": (4096, 14336, 8, 2)}   # (H, I, E, k)
 
-# DRAM bytes (read + write) of one decode FFN call per active expert, from one
-# ncu capture of the gate/up and down GEMV launches at T=16 (57 active
-# experts; gate/up 119.04 MB read + 3.30 MB written, down 59.75 MB read +
-# 0.02 MB written).
-# Reported as roofline.traffic scaled to the bench's active experts; valid
-# while those kernels are the ones captured.
-DECODE_TRAFFIC_PER_ACTIVE_EXPERT = (119.036e6 + 3.302e6 + 59.748e6 + 0.022e6) / 57
+# DRAM bytes (read + write) of one decode FFN call per active expert, from an
+# ncu capture of the shipped gate/up and down kernels at T=16 (None until the
+# current kernels have been captured). Reported as roofline.traffic, scaled to
+# the bench's active experts.
+DECODE_TRAFFIC_PER_ACTIVE_EXPERT = None
+
+# Prefill entries of the default line: (shape, T).
+PREFILL_CASES = (("olmoe", 2048), ("olmoe", 8192), ("wide", 8192))
 
 
 def rec_bytes(h, i):
@@ -63,12 +64,14 @@ def parse():
     ap.add_argument("--T", type=int, default=16)
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="leave the prefill entries out of the default line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc"])
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "slotcache"],
                     help="decode: the 16-layer stack sweep (default); prefill: one layer at large T; "
                          "slotcache: 16 layers decoding from a pinned host pool through S GPU slots per layer")
-    ap.add_argument("--slots", type=int, default=16)
+    ap.add_argument("--slots", default="8,16,32,64",
+                    help="slotcache: slot counts per layer to sweep (comma list); the line's headline is 16")
     ap.add_argument("--shape", default="olmoe", choices=list(SHAPES))
     ap.add_argument("--skew", action="store_true", help="prefill with Zipf(1.2) log-bias routing")
     a = ap.parse_args()
@@ -77,6 +80,14 @@ def parse():
     if a.workload == "prefill" and a.layers == LAYERS:
         a.layers = 1
     return a
+
+
+def decode_config(T, L, world):
+    """The decode workload's config, shared by both arms of the bench."""
+    return {"workload": f"olmoe-{L}L-decode", "T": T, "layers": L, "H": H, "I": I, "E": E, "k": K,
+            "weights": "int4 group-128 symmetric, all experts resident",
+            "l2": "inputs larger than L2 (3.32 GB of packed experts read per step)",
+            "parallelism": f"replicas{world}"}
 
 
 def peaks():
@@ -357,11 +368,12 @@ def run_reference(a):
     if rank != 0:
         return
     v, cores, desc = oracle_sample(a.T, seconds=min(60.0, 2.0 * max(1, a.steps)))
+    # the same workload as the repo arm; the unit is per layer and every layer
+    # has the same shape, so passes of layer 0 are a bounded sample of it
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "layer-tokens/s", "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * a.T * a.layers / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"olmoe-{a.layers}L-decode", "T": a.T, "layers": a.layers, "H": H, "I": I,
-                       "E": E, "k": K},
+            "config": decode_config(a.T, a.layers, a.gpus),
             "cpu_baseline": {"value": v, "unit": "layer-tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": "layer-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -395,6 +407,13 @@ def main():
                              "ffn_hbm_frac": (r["ffn_bytes_per_call"] / (r["ffn_ms_per_call"] / 1e3) / 1e9)
                              / P["hbm_gbs"],
                              "n_active_mean": r["n_active_mean"]}
+    del stack
+    torch.cuda.empty_cache()
+    prefill = {}
+    if not a.no_prefill:
+        for shape, Tp in PREFILL_CASES:
+            prefill[f"{shape}-T{Tp}"] = prefill_entry(a, shape, Tp, rank, world, P)
+            torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         v, cores, desc = oracle_sample(a.T, seconds=10.0)
@@ -410,17 +429,15 @@ def main():
             "metric": METRIC, "value": value, "unit": "layer-tokens/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"olmoe-{L}L-decode", "T": T, "layers": L, "H": H, "I": I, "E": E, "k": K,
-                       "weights": "int4 group-128 symmetric, all experts resident",
-                       "l2": "inputs larger than L2 (3.32 GB of packed experts read per step)",
-                       "parallelism": f"replicas{world}"},
+            "config": decode_config(T, L, world),
             "e2e": {"value": replica_value(T * L, world, head["ms_e2e"]), "unit": "layer-tokens/s",
                     "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
             "roofline": {"bound": "hbm", "kernel": "moe_grouped_w4a16_ffn (gate/up + down kernels), per layer call",
                          "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / P["hbm_gbs"],
                          "traffic": (DECODE_TRAFFIC_PER_ACTIVE_EXPERT * head["n_active_mean"]
-                                     if (T, H, I, E, K) == (16, 2048, 1024, 64, 8) else None),
+                                     if DECODE_TRAFFIC_PER_ACTIVE_EXPERT and (T, H, I, E, K) == (16, 2048, 1024, 64, 8)
+                                     else None),
                          "traffic_source": "ncu capture, scaled by active experts",
                          "peak_source": P["source"], "bytes_per_call": head["ffn_bytes_per_call"],
                          "ms_per_call": head["ffn_ms_per_call"]},
@@ -428,6 +445,7 @@ def main():
             "gpu_launches": head["launches_per_step"] * a.steps,
             "clocks": head["clocks"],
             "sweep": sweep,
+            "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -436,18 +454,27 @@ def main():
         dist.destroy_process_group()
 
 
+# The pages' slot counts (Table 1) and their whole-model L4 hit rates, for context.
+PAGES_HIT_RATE = {8: 0.388, 16: 0.563, 32: 0.814, 64: None}
+
+
 def main_slotcache(a, rank, world, P):
-    """Decode at T=1 with every expert in pinned host memory and `slots` GPU
-    slots per layer; routing drawn so each expert of the previous step is kept
-    with probability 0.5. Each step: per layer, route (weights of the drawn
-    ids), host LRU lookup, H2D fill of the misses on a side stream, group,
-    FFN through the slot table, combine."""
+    """Decode with every expert in pinned host memory and S GPU slots per
+    layer, for each S of --slots (a comma list; the pages' Table 1 sweeps 8,
+    16, 32 and 64 = all experts). T tokens per step (default 1), each an
+    independent routing stream that keeps each expert of its previous step
+    with probability 0.5. Per layer and step: route (weights of the drawn
+    ids), plan the step's experts in cache-sized waves, and per wave: host LRU
+    lookup, H2D fill of the misses on a side stream, grouped FFN through the
+    slot table (that wave's experts only), release; then the combine."""
+    import numpy as np
     import torch
 
     import synth
     M = __import__("w4a16_mixture_experts_moe_b200")
     from w4a16_mixture_experts_moe_b200.layer import LayerBuffers
-    L, S, T = a.layers, a.slots, 1
+    L, T = a.layers, a.T if a.T != 16 else 1
+    slot_counts = [int(v) for v in str(a.slots).split(",")]
     steps = a.steps if a.steps >= 16 else 128
     stack = Stack(L, "auto")
     rec = stack.banks[0].rec
@@ -456,13 +483,12 @@ def main_slotcache(a, rank, world, P):
         pool[l * E * rec:(l + 1) * E * rec].copy_(stack.banks[l].buf)
     stack.banks = None                       # the experts now live only in the pinned pool
     torch.cuda.empty_cache()
-    slots = torch.empty(L * S * rec, dtype=torch.uint8, device="cuda")
-    table = torch.full((L, E), -1, dtype=torch.int32, device="cuda")
-    cache = M.SlotCache(L, E, S, rec, pool, slots, table)
-    routing = [synth.drawn_routing(l, E, K, a.warmup + steps) for l in range(L)]
-    ids_dev = torch.tensor([[routing[l][s] for l in range(L)] for s in range(a.warmup + steps)], dtype=torch.int32,
-                           device="cuda")
-    x0 = synth.activations(a.warmup + steps, H, device="cuda")
+    n_steps = a.warmup + steps
+    # routing[l][s] = ids [T][K] of step s in layer l
+    routing = [np.stack([synth.drawn_routing(l, E, K, n_steps, stream=t) for t in range(T)], axis=1)
+               for l in range(L)]
+    ids_dev = torch.from_numpy(np.stack(routing, axis=1).astype(np.int32)).cuda()   # [step][layer][T][K]
+    x0 = synth.activations(n_steps * T, H, device="cuda").view(n_steps, T, H)
     bufs = [LayerBuffers(T, K, E, H, I) for _ in range(L)]
     xs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     side = torch.cuda.Stream()
@@ -482,61 +508,117 @@ def main_slotcache(a, rank, world, P):
     pinned_gbs = probe_n * rec / (ev0.elapsed_time(ev1) / 1e3) / 1e9
     del dst
 
-    def step(si):
-        cur = x0[si:si + 1]
-        for l in range(L):
-            b = bufs[l]
-            ids = [int(v) for v in routing[l][si]]
-            _, miss = cache.lookup(l, ids)
-            cache.fill(l, miss, side=side, compute=comp)
-            b.topk_ids.copy_(ids_dev[si, l:l + 1])
-            M.moe_route_topk(cur, stack.routers[l], T, H, E, K, None, M.MOE_IDS_GIVEN, b.logits, b.topk_ids,
-                             b.topk_w)
-            M.moe_group_tokens(b.topk_ids, T, K, E, b.counts, b.offsets, b.sorted_pair, b.pair_pos, b.group_ws,
-                               b.group_ws_bytes)
-            M.moe_grouped_w4a16_ffn(cur, b.sorted_pair, b.offsets, slots.data_ptr() + l * S * rec, rec, table[l], S,
-                                    T, K, E, H, I, M.MOE_PATH_AUTO, b.y, b.ffn_ws, b.ffn_ws_bytes)
-            out = xs[l % 2]
-            M.moe_combine(b.y, b.topk_w, b.pair_pos, cur, T, K, H, out)
-            cache.release(l, comp)
-            cur = out
-        return cur
+    def run(S):
+        slots = torch.empty(L * S * rec, dtype=torch.uint8, device="cuda")
+        table = torch.full((L, E), -1, dtype=torch.int32, device="cuda")
+        cache = M.SlotCache(L, E, S, rec, pool, slots, table)
+        n_waves = [0]
 
-    for si in range(a.warmup):
-        step(si)
-    torch.cuda.synchronize()
-    st0 = cache.stats()
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = M.moe_launch_counter()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        s0.record()
-        for si in range(a.warmup, a.warmup + steps):
+        def step(si):
+            cur = x0[si]
+            for l in range(L):
+                b = bufs[l]
+                b.topk_ids.copy_(ids_dev[si, l])
+                M.moe_route_topk(cur, stack.routers[l], T, H, E, K, None, M.MOE_IDS_GIVEN, b.logits, b.topk_ids,
+                                 b.topk_w)
+                M.moe_group_tokens(b.topk_ids, T, K, E, b.counts, b.offsets, b.sorted_pair, b.pair_pos,
+                                   b.group_ws, b.group_ws_bytes)
+                waves = cache.plan_waves(l, [int(v) for v in routing[l][si].reshape(-1)])
+                n_waves[0] += len(waves)
+                for w in waves:
+                    _, miss = cache.lookup(l, w)
+                    cache.fill(l, miss, side=side, compute=comp)
+                    M.moe_grouped_w4a16_ffn(cur, b.sorted_pair, b.offsets, slots.data_ptr() + l * S * rec, rec,
+                                            table[l], S, T, K, E, H, I, M.MOE_PATH_AUTO, b.y, b.ffn_ws,
+                                            b.ffn_ws_bytes)
+                    cache.release(l, comp)
+                out = xs[l % 2]
+                M.moe_combine(b.y, b.topk_w, b.pair_pos, cur, T, K, H, out)
+                cur = out
+            return cur
+
+        for si in range(a.warmup):
             step(si)
-        s1.record()
         torch.cuda.synchronize()
-    launches = M.moe_launch_counter() - launches0
-    ms = s0.elapsed_time(s1) / steps
-    st1 = cache.stats()
-    hits, misses = st1["hits"] - st0["hits"], st1["misses"] - st0["misses"]
-    h2d = st1["h2d_bytes"] - st0["h2d_bytes"]
-    err = [M.moe_read_device_error(b.ffn_ws) for b in bufs]
+        st0 = cache.stats()
+        n_waves[0] = 0
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        launches0 = M.moe_launch_counter()
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            s0.record()
+            for si in range(a.warmup, n_steps):
+                step(si)
+            s1.record()
+            torch.cuda.synchronize()
+        launches = M.moe_launch_counter() - launches0
+        ms = s0.elapsed_time(s1) / steps
+        st1 = cache.stats()
+        hits, misses = st1["hits"] - st0["hits"], st1["misses"] - st0["misses"]
+        h2d = st1["h2d_bytes"] - st0["h2d_bytes"]
+        err = sorted(set(M.moe_read_device_error(b.ffn_ws) for b in bufs))
+        cache.close()
+        del slots, table
+        return {"slots": S, "value": T * L / (ms / 1e3), "unit": "layer-tokens/s", "ms_per_step": ms,
+                "decode_tokens_per_s": T * 1e3 / ms,
+                "hit_rate": None if S >= E else hits / max(1, hits + misses),
+                "pages_hit_rate_l4": PAGES_HIT_RATE.get(S),
+                "h2d_gb": h2d / 1e9, "h2d_gb_per_step": h2d / 1e9 / steps,
+                "h2d_achieved_gbs": h2d / (ms * steps / 1e3) / 1e9,
+                "waves_per_layer_step": n_waves[0] / (steps * L), "device_errors": err,
+                "gpu_launches": launches, "clocks": clk.summary()}
+
+    results = [run(S) for S in slot_counts]
+    head = next((r for r in results if r["slots"] == 16), results[0])
     if rank == 0:
         line = {
-            "metric": METRIC, "value": T * L / (ms / 1e3), "unit": "layer-tokens/s", "n_gpus": world,
-            "steps": steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"olmoe-{L}L-slotcache-decode", "T": T, "layers": L, "slots_per_layer": S,
-                       "H": H, "I": I, "E": E, "k": K, "routing": "drawn, keep-probability 0.5",
+            "metric": METRIC, "value": replica_value(T * L, world, head["ms_per_step"]), "unit": "layer-tokens/s",
+            "n_gpus": world, "steps": steps, "warmup": a.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"olmoe-{L}L-slotcache-decode", "T": T, "layers": L,
+                       "slots_per_layer": head["slots"], "H": H, "I": I, "E": E, "k": K,
+                       "routing": "drawn per token stream, keep-probability 0.5",
                        "pool": f"{L * E * rec / 1e9:.2f} GB pinned host", "parallelism": f"replicas{world}"},
-            "decode_tokens_per_s": 1e3 / ms,
-            "hit_rate": hits / max(1, hits + misses),
-            "h2d_gb": h2d / 1e9, "h2d_gb_per_step": h2d / 1e9 / steps,
-            "h2d_achieved_gbs": h2d / (ms * steps / 1e3) / 1e9, "pinned_copy_gbs": pinned_gbs,
-            "device_errors": sorted(set(err)),
-            "gpu_launches": launches, "clocks": clk.summary(),
+            "decode_tokens_per_s": head["decode_tokens_per_s"], "hit_rate": head["hit_rate"],
+            "h2d_gb": head["h2d_gb"], "h2d_achieved_gbs": head["h2d_achieved_gbs"], "pinned_copy_gbs": pinned_gbs,
+            "device_errors": head["device_errors"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+            "slot_sweep": {str(r["slots"]): r for r in results},
         }
         print(json.dumps(line), flush=True)
-    cache.close()
+
+
+def prefill_entry(a, shape, T, rank, world, P, skew=False):
+    """One prefill layer step (tensor-core path) at T tokens: layer-tokens/s,
+    the grouped FFN call against the BF16 tensor peak, clocks, and the oracle
+    on 64 of the tokens (rank 0, one GPU). Used by the default line."""
+    H_, I_, E_, K_ = SHAPES[shape]
+    renorm = shape == "wide"
+    stack = Stack(1, "auto", shape, renorm=renorm, skew=skew)
+    steps = max(5, min(a.steps, 50))
+    r = measure_T(stack, T, steps, max(3, min(a.warmup, 10)), world)
+    del stack
+    achieved = r["ffn_flops_per_call"] / (r["ffn_ms_per_call"] / 1e3) / 1e12
+    ent = {"value": replica_value(T, world, r["ms_per_step"]), "unit": "layer-tokens/s",
+           "ms_per_step": r["ms_per_step"], "steps": steps,
+           "e2e": {"value": replica_value(T, world, r["ms_e2e"]), "unit": "layer-tokens/s",
+                   "h2d_bytes_per_step": T * H_ * 2, "d2h_bytes_per_step": T * H_ * 2},
+           "config": {"workload": f"{shape}-prefill", "T": T, "layers": 1, "H": H_, "I": I_, "E": E_, "k": K_,
+                      "renorm": renorm,
+                      "l2": f"inputs larger than L2 ({E_ * rec_bytes(H_, I_) / 1e6:.0f} MB of packed experts "
+                            f"+ {T * H_ * 2 / 1e6:.0f} MB of activations)"},
+           "roofline": {"bound": "tensor", "kernel": "moe_grouped_w4a16_ffn (tcgen05 gate/up + down), per call",
+                        "achieved": achieved, "peak": P["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": achieved / P["bf16_tflops"],
+                        "frac_of_sustained": achieved / P["bf16_tflops_sustained"], "traffic": None,
+                        "peak_source": P["source"], "flops_per_call": r["ffn_flops_per_call"],
+                        "ms_per_call": r["ffn_ms_per_call"], "n_active_mean": r["n_active_mean"]},
+           "gpu_launches": r["launches_per_step"] * steps,
+           "clocks": r["clocks"]}
+    ent["cpu_baseline"] = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        v, cores, desc = oracle_sample(T, seconds=5.0, shape=shape, tokens=64, skew=skew, renorm=renorm)
+        ent["cpu_baseline"] = {"value": v, "unit": "layer-tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": desc}
+    return ent
 
 
 def main_prefill(a, rank, world, P):
