@@ -361,6 +361,31 @@ int slot_cache_inject_fill_failure(moe_slot_cache *c, int count);
 
 void slot_cache_destroy(moe_slot_cache *c);
 
+/*
+ * The packed pool as a file: the "quantised and packed once" artifact
+ * (Figure 1 caption: experts are quantised and packed once offline, and the
+ * pinned host pool keeps every packed expert). Host-only calls (no CUDA),
+ * so a pool can be written once and reloaded into pinned memory, a bank or
+ * a slot cache's pool without re-quantising.
+ *   pool    host, [layers][E] records of record_bytes, the layout of a bank
+ *           (records as moe_quantize_pack writes them).
+ * File: a 64-byte little-endian header (magic "EXMOEPK1", format version 1,
+ * header size, layers, E, H, I, record_bytes, payload bytes, and a 64-bit
+ * FNV-1a checksum of the payload taken as little-endian 64-bit words), then
+ * the records. moe_pool_save writes path.tmp and renames it over path.
+ * moe_pool_load checks the header, the shape, the buffer's capacity (bytes),
+ * the file's length and the checksum, and returns MOE_ERR_INVALID_ARG with a
+ * message on any mismatch (MOE_ERR_UNSUPPORTED for another format version).
+ */
+typedef struct {
+  int32_t layers, E, H, I;
+  int64_t record_bytes; /* >= moe_expert_record_layout(H, I).bytes, multiple of 256 */
+} moe_pool_info;
+
+int moe_pool_save(const char *path, const moe_pool_info *info, const void *pool_host);
+int moe_pool_file_info(const char *path, moe_pool_info *info);
+int moe_pool_load(const char *path, void *pool_host, size_t capacity_bytes, moe_pool_info *info);
+
 #ifdef __cplusplus
 }
 #endif

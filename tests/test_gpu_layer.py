@@ -291,3 +291,32 @@ def test_slot_cache_waves_match_oracle(M):
     st = cache.stats()
     assert (st["hits"], st["misses"], st["h2d_bytes"]) == (policy.hits, policy.misses, policy.h2d_bytes(rec))
     cache.close()
+
+
+def test_packed_pool_file_round_trip_runs_the_layer(M, tmp_path):
+    """Pack once on the GPU, save the records to a pool file, load them back
+    into pinned host memory, copy them to a fresh device bank, and run the
+    layer from it: the bank is byte-identical to the packed one, the output
+    bit-identical to the output from the packed bank and within the BF16 bar
+    of the oracle (Figure 1 caption: packed once)."""
+    from w4a16_mixture_experts_moe_b200.layer import ExpertBank, LayerBuffers, moe_layer_forward
+    T = 16
+    bank, wr = _gpu_bank(M, 0)
+    host = bank.buf.cpu()
+    path = str(tmp_path / "olmoe_layer0.pool")
+    M.moe_pool_save(path, 1, E, H, I, bank.rec, host)
+    info = M.moe_pool_file_info(path)
+    assert info == {"layers": 1, "E": E, "H": H, "I": I, "record_bytes": bank.rec}
+    pinned = torch.empty(E * bank.rec, dtype=torch.uint8, pin_memory=True)
+    M.moe_pool_load(path, pinned, pinned.numel())
+    loaded = ExpertBank(E, H, I)
+    loaded.buf.copy_(pinned)
+    assert torch.equal(loaded.buf, bank.buf)
+    x = synth.activations(T, H, seed=81)
+    outs = []
+    for b in (bank, loaded):
+        buf = LayerBuffers(T, K, E, H, I)
+        outs.append((moe_layer_forward(x.cuda(), wr, b, buf).clone(), buf))
+        assert M.moe_read_device_error(buf.ffn_ws) == 0
+    assert torch.equal(outs[0][0], outs[1][0])
+    _run_and_check(M, 0, x, outs[1][1], outs[1][0], "layer from a loaded pool")

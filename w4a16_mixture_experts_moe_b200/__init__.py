@@ -14,6 +14,7 @@ _NATIVE_NAMES = {
     "moe_last_error", "moe_abi_version", "moe_launch_counter", "moe_expert_record_layout", "moe_quantize_pack", "moe_route_topk",
     "moe_group_workspace_size", "moe_group_tokens", "moe_group_tokens_noalloc", "MOE_NOALLOC_MAX_PAIRS", "moe_ffn_workspace_size", "moe_grouped_w4a16_ffn",
     "moe_combine", "moe_read_device_error", "moe_debug_stall_next_tc_ffn", "SlotCache", "MoeError",
+    "moe_pool_save", "moe_pool_file_info", "moe_pool_load",
     "MOE_RENORM", "MOE_LOGITS_GIVEN", "MOE_IDS_GIVEN", "MOE_PATH_AUTO", "MOE_PATH_GEMV", "MOE_PATH_TC", "MOE_SLOT_SKIP",
     "MOE_DEVERR_NONE", "MOE_DEVERR_EXPERT_ID", "MOE_DEVERR_NOT_RESIDENT", "MOE_DEVERR_TIMEOUT", "MOE_DEVERR_RANGE",
 }

@@ -38,6 +38,11 @@ class moe_record_layout(C.Structure):
                 ("gate_s", _i64), ("up_s", _i64), ("down_s", _i64), ("bytes", _i64)]
 
 
+class moe_pool_info(C.Structure):
+    _fields_ = [("layers", C.c_int32), ("E", C.c_int32), ("H", C.c_int32), ("I", C.c_int32),
+                ("record_bytes", _i64)]
+
+
 # name -> (restype, argtypes); kept in the order of include/exactmoe.h
 SIGNATURES = {
     "moe_last_error": (C.c_char_p, []),
@@ -62,6 +67,9 @@ SIGNATURES = {
     "slot_cache_stats": (_i, [_p, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]),
     "slot_cache_inject_fill_failure": (_i, [_p, _i]),
     "slot_cache_destroy": (None, [_p]),
+    "moe_pool_save": (_i, [C.c_char_p, C.POINTER(moe_pool_info), _p]),
+    "moe_pool_file_info": (_i, [C.c_char_p, C.POINTER(moe_pool_info)]),
+    "moe_pool_load": (_i, [C.c_char_p, _p, _sz, C.POINTER(moe_pool_info)]),
 }
 
 for _name, (_res, _args) in SIGNATURES.items():
@@ -234,3 +242,28 @@ class SlotCache:
             self.close()
         except Exception:
             pass
+
+
+def _info_dict(info):
+    return {f: getattr(info, f) for f, _ in moe_pool_info._fields_}
+
+
+def moe_pool_save(path, layers, E, H, I, record_bytes, pool):
+    """Writes the host pool (a tensor, numpy array via its address, or int) to path."""
+    info = moe_pool_info(layers, E, H, I, record_bytes)
+    addr = pool if isinstance(pool, int) else (pool.ctypes.data if hasattr(pool, "ctypes") else pool.data_ptr())
+    _check(lib.moe_pool_save(os.fsencode(path), C.byref(info), addr))
+
+
+def moe_pool_file_info(path) -> dict:
+    info = moe_pool_info()
+    _check(lib.moe_pool_file_info(os.fsencode(path), C.byref(info)))
+    return _info_dict(info)
+
+
+def moe_pool_load(path, pool, capacity) -> dict:
+    """Reads path's records into the host buffer `pool` of `capacity` bytes."""
+    info = moe_pool_info()
+    addr = pool if isinstance(pool, int) else (pool.ctypes.data if hasattr(pool, "ctypes") else pool.data_ptr())
+    _check(lib.moe_pool_load(os.fsencode(path), addr, capacity, C.byref(info)))
+    return _info_dict(info)
