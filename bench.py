@@ -65,8 +65,10 @@ def parse():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="leave the prefill entries out of the default line")
+    ap.add_argument("--no-references", action="store_true",
+                    help="leave the sequential-W4 and BF16 reference paths out of the default line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc"])
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc", "seq"])
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "slotcache"],
                     help="decode: the 16-layer stack sweep (default); prefill: one layer at large T; "
                          "slotcache: 16 layers decoding from a pinned host pool through S GPU slots per layer")
@@ -217,7 +219,8 @@ class Stack:
         self.flags = M.MOE_RENORM if renorm else 0
         # skewed routing: log Zipf(1.2) per-expert offsets added to the logits
         self.bias = torch.from_numpy(synth.zipf_log_bias(E)).float().cuda() if skew else None
-        self.path = {"auto": M.MOE_PATH_AUTO, "gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC}[path]
+        self.path = {"auto": M.MOE_PATH_AUTO, "gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC,
+                     "seq": M.MOE_PATH_SEQUENTIAL}[path]
         self.banks, self.routers = [], []
         for l in range(layers):
             gate, up, down = synth.expert_bank(l, E, H, I, device="cuda")
@@ -407,6 +410,9 @@ def main():
                              "ffn_hbm_frac": (r["ffn_bytes_per_call"] / (r["ffn_ms_per_call"] / 1e3) / 1e9)
                              / P["hbm_gbs"],
                              "n_active_mean": r["n_active_mean"]}
+    refs = {}
+    if not a.no_references:
+        refs = reference_paths(a, stack, head, world, P)
     del stack
     torch.cuda.empty_cache()
     prefill = {}
@@ -446,6 +452,7 @@ def main():
             "clocks": head["clocks"],
             "sweep": sweep,
             "prefill": prefill,
+            "references": refs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -584,6 +591,94 @@ def main_slotcache(a, rank, world, P):
             "slot_sweep": {str(r["slots"]): r for r in results},
         }
         print(json.dumps(line), flush=True)
+
+
+# The pages' own ratios for these two comparisons, measured on one L4 on the
+# whole OLMoE model (context only): fused grouped execution against the
+# sequential W4 reference at 16 tokens, and W4A16 against BF16 decode.
+PAGES_FUSED_OVER_SEQUENTIAL_L4 = 1.97
+PAGES_W4_OVER_BF16_DECODE_L4 = 31.923 / 21.662
+
+
+def reference_paths(a, stack, head, world, P):
+    """The decode step at the bench's T through the two reference paths the
+    pages compare against: the sequential W4 reference (the same GEMV kernels
+    launched once per expert, MOE_PATH_SEQUENTIAL) and the BF16 grouped FFN
+    on unquantised experts (moe_grouped_bf16_ffn; 12.6 MB per OLMoE expert,
+    12.9 GB for the 16 layers). Route, group and combine are the same calls in
+    all three; each step is replayed from a CUDA graph."""
+    import torch
+
+    import synth
+    from w4a16_mixture_experts_moe_b200.layer import Bf16Bank
+    M, T, L = stack.M, a.T, stack.layers
+    steps = max(5, min(a.steps, 50))
+    old = stack.path
+    stack.path = M.MOE_PATH_SEQUENTIAL
+    r = measure_T(stack, T, steps, a.warmup, world, want_e2e=False)
+    stack.path = old
+    seq = {"ms_per_step": r["ms_per_step"], "value": replica_value(T * L, world, r["ms_per_step"]),
+           "unit": "layer-tokens/s", "ffn_ms_per_call": r["ffn_ms_per_call"],
+           "launches_per_step": r["launches_per_step"],
+           "fused_over_sequential_step": r["ms_per_step"] / head["ms_per_step"],
+           "fused_over_sequential_ffn": r["ffn_ms_per_call"] / head["ffn_ms_per_call"],
+           "pages_fused_over_sequential_l4": PAGES_FUSED_OVER_SEQUENTIAL_L4}
+
+    banks = []
+    for l in range(L):
+        g, u, d = synth.expert_bank(l, E, H, I, device="cuda")
+        b = Bf16Bank(E, H, I)
+        b.load(g, u, d)
+        del g, u, d
+        banks.append(b)
+    bufs, xs = stack.buffers(T)
+    nb = M.moe_bf16_ffn_workspace_size(T, K, E, H, I)
+    wss = [torch.zeros(nb, dtype=torch.uint8, device="cuda") for _ in range(L)]
+    x_in = synth.activations(T, H, device="cuda")
+
+    def ffn(l, cur):
+        bb = bufs[l]
+        M.moe_grouped_bf16_ffn(cur, bb.sorted_pair, bb.offsets, banks[l].ptr, banks[l].rec, T, K, E, H, I, bb.y,
+                               wss[l], nb)
+
+    def fwd():
+        cur = x_in
+        for l in range(L):
+            bb = bufs[l]
+            out = xs[l % 2] if cur is not xs[l % 2] else xs[(l + 1) % 2]
+            M.moe_route_topk(cur, stack.routers[l], T, H, E, K, None, 0, bb.logits, bb.topk_ids, bb.topk_w)
+            M.moe_group_tokens(bb.topk_ids, T, K, E, bb.counts, bb.offsets, bb.sorted_pair, bb.pair_pos,
+                               bb.group_ws, bb.group_ws_bytes)
+            ffn(l, cur)
+            M.moe_combine(bb.y, bb.topk_w, bb.pair_pos, cur, T, K, H, out)
+            cur = out
+        return cur
+
+    fwd()
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        fwd()
+    ms = max_over_ranks(time_graph(torch, g1, steps, a.warmup), world)
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        cur = x_in
+        for l in range(L):
+            ffn(l, x_in if l == 0 else xs[(l - 1) % 2])
+    ms_ffn = time_graph(torch, g2, steps, 3) / L
+    n_act = statistics.mean(int((b.counts > 0).sum().item()) for b in bufs)
+    bf16_bytes = n_act * banks[0].rec
+    del g1, g2, banks
+    torch.cuda.empty_cache()
+    bf = {"ms_per_step": ms, "value": replica_value(T * L, world, ms), "unit": "layer-tokens/s",
+          "ffn_ms_per_call": ms_ffn, "n_active_mean": n_act, "ffn_bytes_per_call": bf16_bytes,
+          "ffn_hbm_frac": bf16_bytes / (ms_ffn / 1e3) / 1e9 / P["hbm_gbs"],
+          "w4_over_bf16_step": ms / head["ms_per_step"],
+          "w4_over_bf16_ffn": ms_ffn / head["ffn_ms_per_call"],
+          "pages_w4_over_bf16_decode_l4": PAGES_W4_OVER_BF16_DECODE_L4}
+    return {"T": T, "sequential_w4": seq, "bf16_grouped": bf}
 
 
 def prefill_entry(a, shape, T, rank, world, P, skew=False):

@@ -203,6 +203,9 @@ int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E,
 #define MOE_PATH_AUTO 0 /* chosen from the average rows per expert, T*k/E */
 #define MOE_PATH_GEMV 1 /* decode-sized groups: weight-streaming, HBM-bound */
 #define MOE_PATH_TC 2   /* prefill-sized groups: tcgen05 tensor cores */
+#define MOE_PATH_SEQUENTIAL 3 /* reference only: the GEMV kernels launched
+                                 once per expert, expert after expert (the
+                                 pages' sequential W4 baseline, Abstract) */
 
 /*
  * A5 + A6 — the grouped SwiGLU expert FFN with in-kernel int4 dequantisation
@@ -248,6 +251,31 @@ int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pair,
                           int n_slots, int T, int k, int E, int H, int I,
                           int path, float *y, void *ws, size_t ws_bytes,
                           moe_stream_t stream);
+
+/*
+ * The BF16 grouped expert FFN (the pages' BF16 baseline, Abstract and
+ * Table 1): the same grouped SwiGLU with unquantised BF16 experts, for
+ * measuring what the int4 packing buys. Not part of the W4A16 path.
+ * A BF16 record holds gate [I][H], up [I][H] and down [H][I] BF16 weights
+ * (nn.Linear layout) at the offsets moe_bf16_record_layout gives (multiples
+ * of 256). For sorted row r of expert e and token t = sorted_pair[r] / k:
+ *   h[r] = bf16_rn(silu(x[t] Wg_e^T) * (x[t] Wu_e^T))  (fp32 sums, h in BF16)
+ *   y[r] = h[r] Wd_e^T                                  (fp32 sums, fp32)
+ * Arguments as moe_grouped_w4a16_ffn (identity expert -> record mapping);
+ * ws holds the error word and h.
+ */
+typedef struct {
+  int64_t gate, up, down; /* byte offsets of the three matrices */
+  int64_t bytes;          /* record size */
+} moe_bf16_layout;
+
+int moe_bf16_record_layout(int H, int I, moe_bf16_layout *out);
+size_t moe_bf16_ffn_workspace_size(int T, int k, int E, int H, int I);
+int moe_grouped_bf16_ffn(const moe_bf16 *x, const int32_t *sorted_pair,
+                         const int32_t *offsets, const void *bank,
+                         int64_t record_bytes, int T, int k, int E, int H,
+                         int I, float *y, void *ws, size_t ws_bytes,
+                         moe_stream_t stream);
 
 /*
  * Test hook for the failure path of the tensor-core FFN: the next `calls`

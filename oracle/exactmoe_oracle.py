@@ -306,6 +306,18 @@ class LazyQuantizedExperts:
         return self._cache(int(e))
 
 
+class Bf16Experts:
+    """Unquantised experts, the pages' BF16 baseline (Abstract and Table 1
+    compare the W4A16 model with the BF16 one): weights_of(e) returns expert
+    e's BF16-valued (gate [I][H], up [I][H], down [H][I]), used as they are."""
+
+    def __init__(self, weights_of, E: int, H: int, I: int):
+        self.weights_of, self.E, self.H, self.I = weights_of, E, H, I
+
+    def dequantized(self, e: int):
+        return tuple(np.asarray(w, dtype=np.float64) for w in self.weights_of(int(e)))
+
+
 def grouped_ffn(x, experts: PackedExperts, sorted_pair, offsets, k: int):
     """Grouped form: per expert, its rows in sorted order.
 

@@ -213,12 +213,13 @@ def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None):
     return y.cpu().double().numpy(), h.float().cpu().double().numpy(), code
 
 
-@pytest.mark.parametrize("path", ["gemv", "tc"])
+@pytest.mark.parametrize("path", ["gemv", "tc", "seq"])
 @pytest.mark.parametrize("E,H,I,T,k", [(5, 256, 384, 13, 2), (4, 512, 256, 40, 3), (64, 2048, 1024, 16, 8),
                                        (8, 4096, 1024, 9, 2), (4, 512, 256, 300, 2), (6, 384, 640, 700, 3),
                                        (64, 2048, 1024, 1, 8), (64, 2048, 1024, 64, 8)])
 def test_grouped_ffn(M, path, E, H, I, T, k):
-    P = {"gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC}[path]
+    """Both FFN paths, and the sequential per-expert reference, against the oracle."""
+    P = {"gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC, "seq": M.MOE_PATH_SEQUENTIAL}[path]
     rng = np.random.default_rng(E * H + T)
     gate = synth.normal_bf16((E, I, H), 0.02, 1000 + E)
     up = synth.normal_bf16((E, I, H), 0.02, 2000 + E)
@@ -233,6 +234,40 @@ def test_grouped_ffn(M, path, E, H, I, T, k):
     ref_h, ref_y = o.grouped_ffn(x.double().numpy(), experts, sp, offsets, k)
     assert_bf16_close(h, ref_h, "h")
     assert_bf16_close(y, ref_y, "y")
+
+
+@pytest.mark.parametrize("E,H,I,T,k", [(5, 256, 384, 13, 2), (64, 2048, 1024, 16, 8), (8, 4096, 1024, 9, 2),
+                                       (4, 512, 256, 300, 2), (64, 2048, 1024, 1, 8)])
+def test_grouped_bf16_ffn(M, E, H, I, T, k):
+    """The BF16 baseline: unquantised experts through moe_grouped_bf16_ffn
+    against the oracle's grouped FFN on the same BF16 weights."""
+    from w4a16_mixture_experts_moe_b200.layer import Bf16Bank
+    rng = np.random.default_rng(E * H + T + 1)
+    gate = synth.normal_bf16((E, I, H), 0.02, 1100 + E)
+    up = synth.normal_bf16((E, I, H), 0.02, 2100 + E)
+    down = synth.normal_bf16((E, H, I), 0.02, 3100 + E)
+    x = synth.activations(T, H, seed=6)
+    ids = np.stack([rng.choice(E - 1, size=k, replace=False) for _ in range(T)]).astype(np.int32)  # expert E-1 empty
+    bank = Bf16Bank(E, H, I)
+    bank.load(gate.cuda(), up.cuda(), down.cuda())
+    d = torch.from_numpy(ids).cuda()
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    sp = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    pp = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    gws = torch.zeros(M.moe_group_workspace_size(T, k, E), dtype=torch.uint8, device="cuda")
+    M.moe_group_tokens(d, T, k, E, counts, offsets, sp, pp, gws, gws.numel())
+    y = torch.full((T * k, H), float("nan"), dtype=torch.float32, device="cuda")
+    nb = M.moe_bf16_ffn_workspace_size(T, k, E, H, I)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    M.moe_grouped_bf16_ffn(x.cuda(), sp, offsets, bank.ptr, bank.rec, T, k, E, H, I, y, ws, nb)
+    torch.cuda.synchronize()
+    h = ws[256:256 + T * k * I * 2].view(torch.bfloat16).view(T * k, I).double().cpu().numpy()
+    experts = o.Bf16Experts(torch_weights_source(gate, up, down), E, H, I)
+    _, o_off, o_sp, _ = o.group_tokens(ids, E)
+    ref_h, ref_y = o.grouped_ffn(x.double().numpy(), experts, o_sp, o_off, k)
+    assert_bf16_close(h, ref_h, "bf16 h")
+    assert_bf16_close(y.cpu().double().numpy(), ref_y, "bf16 y")
 
 
 def test_grouped_ffn_not_resident_is_flagged(M):

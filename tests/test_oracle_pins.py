@@ -267,6 +267,29 @@ def test_single_expert_top1_equals_dense_swiglu():
     assert np.array_equal(out, ref)
 
 
+def test_bf16_experts_top1_equals_dense_swiglu():
+    # the BF16 baseline's experts are used unquantised: with one expert and
+    # k = 1 the layer is a dense SwiGLU on the raw weights (torch), h rounded
+    # to BF16, the output rounded to BF16
+    rng = np.random.default_rng(21)
+    T, H, I = 5, 256, 128
+    x = _bf16_values(rng, (T, H), 1.0)
+    wg, wu = _bf16_values(rng, (I, H), 0.05), _bf16_values(rng, (I, H), 0.05)
+    wd = _bf16_values(rng, (H, I), 0.05)
+    ex = o.Bf16Experts(lambda e: (wg, wu, wd), 1, H, I)
+    ids = np.zeros((T, 1), dtype=np.int32)
+    out = o.moe_layer_grouped(x, ex, ids, np.ones((T, 1)))
+    xt = torch.from_numpy(x)
+    g = torch.nn.functional.linear(xt, torch.from_numpy(wg))
+    u = torch.nn.functional.linear(xt, torch.from_numpy(wu))
+    h = (torch.nn.functional.silu(g) * u).to(torch.bfloat16).double()
+    ref = torch.nn.functional.linear(h, torch.from_numpy(wd)).to(torch.bfloat16).double().numpy()
+    assert np.mean(out == ref) > 0.99 and np.allclose(out, ref, rtol=2.0 ** -7, atol=1e-6)
+    # and it differs from the quantised experts' layer on the same weights
+    q = o.LazyQuantizedExperts(lambda e: (wg, wu, wd), 1, H, I)
+    assert not np.array_equal(out, o.moe_layer_grouped(x, q, ids, np.ones((T, 1))))
+
+
 def test_per_token_loop_equals_grouped_form():
     rng = np.random.default_rng(9)
     T, H, I, E, k = 24, 256, 128, 6, 2

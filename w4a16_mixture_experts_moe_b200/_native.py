@@ -24,7 +24,7 @@ lib = C.CDLL(LIB_PATH)
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE, MOE_ERR_CUDA, MOE_ERR_CAPACITY, MOE_ERR_DEVICE, MOE_ERR_UNSUPPORTED = range(7)
 MOE_DEVERR_NONE, MOE_DEVERR_EXPERT_ID, MOE_DEVERR_NOT_RESIDENT, MOE_DEVERR_TIMEOUT, MOE_DEVERR_RANGE = range(5)
 MOE_RENORM, MOE_LOGITS_GIVEN, MOE_IDS_GIVEN = 1, 2, 4
-MOE_PATH_AUTO, MOE_PATH_GEMV, MOE_PATH_TC = 0, 1, 2
+MOE_PATH_AUTO, MOE_PATH_GEMV, MOE_PATH_TC, MOE_PATH_SEQUENTIAL = 0, 1, 2, 3
 MOE_SLOT_SKIP = -2
 
 _p = C.c_void_p
@@ -36,6 +36,10 @@ _sz = C.c_size_t
 class moe_record_layout(C.Structure):
     _fields_ = [("gate_q", _i64), ("up_q", _i64), ("down_q", _i64),
                 ("gate_s", _i64), ("up_s", _i64), ("down_s", _i64), ("bytes", _i64)]
+
+
+class moe_bf16_layout(C.Structure):
+    _fields_ = [("gate", _i64), ("up", _i64), ("down", _i64), ("bytes", _i64)]
 
 
 class moe_pool_info(C.Structure):
@@ -56,6 +60,9 @@ SIGNATURES = {
     "moe_group_tokens_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
     "moe_ffn_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moe_grouped_w4a16_ffn": (_i, [_p, _p, _p, _p, _i64, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "moe_bf16_record_layout": (_i, [_i, _i, C.POINTER(moe_bf16_layout)]),
+    "moe_bf16_ffn_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "moe_grouped_bf16_ffn": (_i, [_p, _p, _p, _p, _i64, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "moe_debug_stall_next_tc_ffn": (_i, [_i]),
     "moe_combine": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_read_device_error": (_i, [_p, _p, C.POINTER(C.c_int32)]),
@@ -165,6 +172,22 @@ def moe_grouped_w4a16_ffn(x, sorted_pair, offsets, bank, record_bytes, expert_sl
     _check(lib.moe_grouped_w4a16_ffn(_ptr(x), _ptr(sorted_pair), _ptr(offsets), _ptr(bank), record_bytes,
                                      _ptr(expert_slot), n_slots, T, k, E, H, I, path, _ptr(y), _ptr(ws), ws_bytes,
                                      _stream(stream)))
+
+
+def moe_bf16_record_layout(H: int, I: int) -> dict:
+    out = moe_bf16_layout()
+    _check(lib.moe_bf16_record_layout(H, I, C.byref(out)))
+    return {f: getattr(out, f) for f, _ in moe_bf16_layout._fields_}
+
+
+def moe_bf16_ffn_workspace_size(T, k, E, H, I) -> int:
+    return lib.moe_bf16_ffn_workspace_size(T, k, E, H, I)
+
+
+def moe_grouped_bf16_ffn(x, sorted_pair, offsets, bank, record_bytes, T, k, E, H, I, y, ws, ws_bytes,
+                         stream=None):
+    _check(lib.moe_grouped_bf16_ffn(_ptr(x), _ptr(sorted_pair), _ptr(offsets), _ptr(bank), record_bytes, T, k, E,
+                                    H, I, _ptr(y), _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def moe_debug_stall_next_tc_ffn(calls: int):

@@ -113,7 +113,7 @@ namespace moe {
 // fallback to the GEMV path on other hardware).
 static bool may_use_tc(int T, int k, int E, int path) {
   if (path == MOE_PATH_TC) return true;
-  if (path == MOE_PATH_GEMV) return false;
+  if (path == MOE_PATH_GEMV || path == MOE_PATH_SEQUENTIAL) return false;
   return int64_t(T) * k >= int64_t(TC_MIN_ROWS_PER_EXPERT) * E;
 }
 }  // namespace moe
@@ -137,7 +137,7 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
     return set_error(MOE_ERR_SHAPE, "moe_grouped_w4a16_ffn: H=%d I=%d must be positive multiples of 128", H, I);
   if (int64_t(T) * k > (int64_t(1) << 30))
     return set_error(MOE_ERR_SHAPE, "moe_grouped_w4a16_ffn: T*k too large");
-  if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_TC)
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_TC && path != MOE_PATH_SEQUENTIAL)
     return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: unknown path %d", path);
   moe_record_layout L;
   int st = moe_expert_record_layout(H, I, &L);
@@ -170,7 +170,9 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
   a.xs = a.x16;
   a.y = y;
   a.stall = 0;
+  a.e0 = 0;
   if (T == 0) return MOE_OK;
+  if (path == MOE_PATH_SEQUENTIAL) return launch_ffn_sequential(a, s);
 
   if (may_use_tc(T, k, E, path)) {
     a.stall = take_tc_stall();

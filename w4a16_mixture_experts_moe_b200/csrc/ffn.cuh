@@ -25,6 +25,7 @@ struct FfnArgs {
   float *y;       // [P][H] fp32 expert outputs, sorted order
   int32_t *err;   // device error word
   int stall;      // test hook: producers never publish a stage (bounded waits run out)
+  int e0;         // first expert of the launch (blockIdx.y + e0; the sequential path launches one expert)
 };
 
 // Test hook state (moe_debug_stall_next_tc_ffn): number of tensor-core FFN
@@ -46,6 +47,7 @@ __device__ __forceinline__ const uint8_t *expert_record(const FfnArgs &a, int e)
 int launch_x_to_f16(const FfnArgs &a, cudaStream_t s);
 int launch_gather_x_f16(const FfnArgs &a, cudaStream_t s);
 int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s);
+int launch_ffn_sequential(const FfnArgs &a, cudaStream_t s);
 int launch_ffn_tc(const FfnArgs &a, cudaStream_t s);
 
 }  // namespace moe

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
   __shared__ uint4 rings[GV_WARPS][GV_DEPTH_GATEUP * 8 * 32];  // [slot][gate g, g+8, g+16, g+24, up ...][lane]
   pdl_trigger();
   pdl_wait();
-  const int e = blockIdx.y;
+  const int e = blockIdx.y + a.e0;
   const int lo = a.offsets[e], cnt = a.offsets[e + 1] - lo;
   if (cnt <= 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
   __shared__ uint4 rings[GV_WARPS][GV_DEPTH_DOWN * 4 * 32];  // [slot][rows g, g+8, g+16, g+24][lane]
   pdl_trigger();
   pdl_wait();
-  const int e = blockIdx.y;
+  const int e = blockIdx.y + a.e0;
   const int lo = a.offsets[e], cnt = a.offsets[e + 1] - lo;
   if (cnt <= 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -375,6 +375,34 @@ static int pick_ksplit(const FfnArgs &a) {
   // warps per slice shorten each CTA's life enough to pay for the reduction
   const bool many_rows = int64_t(a.T) * a.k >= 4 * int64_t(a.E);
   return warps * 2 <= want ? 4 : (warps * 1.25 <= want || many_rows ? 2 : 1);
+}
+
+// The sequential reference (the pages' "sequential W4" baseline, Abstract):
+// the same kernels launched once per expert, gate/up then down, expert after
+// expert, each launch covering one expert's rows with the widest K split.
+// Experts without rows still get their (empty) launches: the host does not
+// know the group sizes without a synchronisation.
+int launch_ffn_sequential(const FfnArgs &a, cudaStream_t s) {
+  int st = launch_x_to_f16(a, s);
+  if (st != MOE_OK) return st;
+  constexpr int KS = 4;
+  const int rows_per_cta = (GV_WARPS / KS) * 16;
+  for (int e = 0; e < a.E; ++e) {
+    FfnArgs b = a;
+    b.e0 = e;
+    cudaError_t err =
+        launch_pdl(gemv_gateup_kernel<KS>, dim3((a.I + rows_per_cta * 2 - 1) / (rows_per_cta * 2), 1),
+                   dim3(GV_WARPS * 32), 0, s, b);
+    if (err == cudaSuccess) {
+      count_launches(1);
+      err = launch_pdl(gemv_down_kernel<KS>, dim3((a.H + rows_per_cta * 2 - 1) / (rows_per_cta * 2), 1),
+                       dim3(GV_WARPS * 32), 0, s, b);
+    }
+    if (err != cudaSuccess)
+      return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (sequential): %s", cudaGetErrorString(err));
+    count_launches(1);
+  }
+  return check_launch("moe_grouped_w4a16_ffn (sequential)", 0);
 }
 
 int launch_ffn_gemv(const FfnArgs &a, cudaStream_t s) {

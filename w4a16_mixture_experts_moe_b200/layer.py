@@ -53,6 +53,30 @@ class ExpertBank:
         return self.buf[off:off + rows * cols // 128 * 2].view(torch.int16).view(rows, cols // 128)
 
 
+class Bf16Bank:
+    """A device array of unquantised BF16 expert records (the BF16 baseline's
+    weights): `load` copies gate, up [E][I][H] and down [E][H][I] BF16 tensors
+    into the records at the offsets moe_bf16_record_layout gives."""
+
+    def __init__(self, n_records: int, H: int, I: int, device="cuda"):
+        self.H, self.I, self.n = H, I, n_records
+        self.layout = N.moe_bf16_record_layout(H, I)
+        self.rec = self.layout["bytes"]
+        self.buf = torch.empty(n_records * self.rec, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    def load(self, gate, up, down, first: int = 0):
+        E = gate.shape[0]
+        recs = self.buf[first * self.rec:(first + E) * self.rec].view(E, self.rec)
+        for w, part in ((gate, "gate"), (up, "up"), (down, "down")):
+            n = w[0].numel() * 2
+            off = self.layout[part]
+            recs[:, off:off + n].copy_(w.contiguous().view(E, -1).view(torch.uint8))
+
+
 class LayerBuffers:
     """Per-shape device buffers of one layer step (T tokens, top-k of E)."""
 
