@@ -216,7 +216,8 @@ def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None):
 @pytest.mark.parametrize("path", ["gemv", "tc", "seq"])
 @pytest.mark.parametrize("E,H,I,T,k", [(5, 256, 384, 13, 2), (4, 512, 256, 40, 3), (64, 2048, 1024, 16, 8),
                                        (8, 4096, 1024, 9, 2), (4, 512, 256, 300, 2), (6, 384, 640, 700, 3),
-                                       (64, 2048, 1024, 1, 8), (64, 2048, 1024, 64, 8)])
+                                       (64, 2048, 1024, 1, 8), (64, 2048, 1024, 64, 8),
+                                       (8, 1024, 1024, 40, 2), (4, 1024, 2048, 100, 2)])
 def test_grouped_ffn(M, path, E, H, I, T, k):
     """Both FFN paths, and the sequential per-expert reference, against the oracle."""
     P = {"gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC, "seq": M.MOE_PATH_SEQUENTIAL}[path]

@@ -1,8 +1,9 @@
 // A5 + A6, decode-sized groups: a weight-streaming grouped GEMV on the
 // warp-level tensor-core MMA (mma.sync m16n8k16, FP16 in, fp32 out).
 //
-// A warp owns 32 output rows of one expert (two 16-row slices side by side)
-// and walks K one 128-wide quantisation group at a time. Lane (g, t) =
+// A warp owns 32 (gate/up: two 16-row slices of both matrices) or 64 (down:
+// four slices) output rows of one expert and walks K one 128-wide
+// quantisation group at a time. Lane (g, t) =
 // (lane/4, lane%4) copies 16 bytes (32 codes) of rows g, g+8, g+16 and g+24
 // per matrix: the group's four lanes read 64 contiguous bytes of each row.
 // The codes never leave registers once read: each packed word turns into four
@@ -12,14 +13,13 @@
 // fragment's k order); the B fragment (the tokens' activations, FP16 copies,
 // or h in the down pass) is loaded with the same binding, so lane t reads 64
 // contiguous bytes of each token row, and one B fragment feeds every MMA tile
-// of the warp (four in gate/up, two in down). The fp32 sum of q*x over one
+// of the warp (four in gate/up and in down). The fp32 sum of q*x over one
 // group is then multiplied by that row's group scale, so the dequantised
 // weight q*s is never rounded.
 //
 // The codes stream through a per-warp shared-memory ring filled by cp.async,
-// DEPTH - 1 groups ahead of the math (gate/up: 4 KB slots, 2 deep; down: 2 KB
-// slots, 4 deep), while each group's B fragment and scales are loaded one
-// group ahead into registers. Each lane copies, and later reads back, only its
+// DEPTH - 1 groups ahead of the math (4 KB slots, 2 deep), while each group's
+// B fragment and scales are loaded one group ahead into registers. Each lane copies, and later reads back, only its
 // own 16-byte pieces, so its own cp.async waits suffice.
 //
 // Why FP16 operands: unpacking codes costs integer instructions, and FP16's
@@ -36,7 +36,7 @@
 namespace moe {
 
 constexpr int GV_WARPS = 4;  // per CTA: 128 rows, or 128 / KS with a K split
-constexpr int GV_DEPTH_DOWN = 4;    // down: ring slots (groups of codes) per warp, 2 KB each
+constexpr int GV_DEPTH_DOWN = 2;    // down: ring slots (groups of codes) per warp, 4 KB each
 constexpr int GV_DEPTH_GATEUP = 2;  // gate/up: ring slots per warp, 4 KB each
 
 // 16-byte asynchronous copy global -> shared, cached in L2 only.
@@ -45,6 +45,21 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
                "l"(src)
                : "memory");
 }
+// The same copy with an L2 eviction-priority policy from createpolicy.
+__device__ __forceinline__ void cp_async16_hint(void *dst, const void *src, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "l"(policy)
+               : "memory");
+}
+// Codes are read exactly once per call: marking them evict-first keeps the
+// small, reused data (activations, h, scales) resident in L2 instead.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -130,6 +145,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
   const bool rows_ok = row0 < a.I;  // I is a multiple of 128, so then all 32 rows are
   const uint8_t *rec = expert_record(a, e);
   if (!rec) return;
+  const uint64_t stream_policy = l2_evict_first_policy();
   const int H = a.H, KB = H / 2, G = H / GROUP;
   const int rr = rows_ok ? row0 + g : 0;
   const uint8_t *gq0 = rec + a.off_gq + int64_t(rr) * KB + t * 16;
@@ -149,8 +165,8 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
       uint4 *d = ring + (i % GV_DEPTH_GATEUP) * (8 * 32) + lane;
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        cp_async16(d + 32 * r, gq0 + r * 8 * KB + grp * 64);
-        cp_async16(d + 128 + 32 * r, uq0 + r * 8 * KB + grp * 64);
+        cp_async16_hint(d + 32 * r, gq0 + r * 8 * KB + grp * 64, stream_policy);
+        cp_async16_hint(d + 128 + 32 * r, uq0 + r * 8 * KB + grp * 64, stream_policy);
       }
     };
 #pragma unroll
@@ -238,27 +254,29 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_gateup_kernel(const FfnArg
   }
 }
 
-// down: y[r][row] = h[r] . Wd[row] (fp32). A warp owns 32 output rows (two
-// 16-row slices side by side): per 128-wide group it copies 16 bytes of rows
-// g, g+8, g+16 and g+24 (2 KB per warp, as in the gate/up pass) and runs both
-// slices' MMAs on the same h fragment, which it loads one group ahead with
-// the group's scales. KS warps split the groups of a slice pair as in the
-// gate/up pass. (One 16-row slice per warp, half the bytes per h fragment,
-// measured 3-10 % slower.)
+// down: y[r][row] = h[r] . Wd[row] (fp32). A warp owns DOWN_RS = 4 16-row
+// slices side by side (64 output rows): per 128-wide group it copies 16 bytes
+// of each of its rows g + 8j (4 KB per warp) and runs all four slices' MMAs
+// on the same h fragment, which it loads one group ahead with the group's
+// scales. KS warps split the groups of a slice set as in the gate/up pass.
+// (Two slices per warp with a 4-deep ring measured 5 % slower at T = 16, one
+// slice per warp 3-10 % slower still.)
+constexpr int DOWN_RS = 4;
 template <int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs a) {
-  __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][8][32];
-  __shared__ uint4 rings[GV_WARPS][GV_DEPTH_DOWN * 4 * 32];  // [slot][rows g, g+8, g+16, g+24][lane]
+  constexpr int RS = DOWN_RS, NP = 2 * RS, DEPTH = GV_DEPTH_DOWN;  // NP: 16-byte pieces per lane per group
+  __shared__ float red[KS > 1 ? KS - 1 : 1][GV_WARPS / KS][KS > 1 ? 4 * RS : 1][32];
+  __shared__ uint4 rings[GV_WARPS][DEPTH * NP * 32];  // [slot][piece: rows g, g+8, g+16, ...][lane]
   pdl_trigger();
   pdl_wait();
   const int e = blockIdx.y + a.e0;
   const int lo = a.offsets[e], cnt = a.offsets[e + 1] - lo;
   if (cnt <= 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int sl = warp / KS, kq = warp % KS;  // slice pair within the CTA, K part
-  const int row0 = (blockIdx.x * (GV_WARPS / KS) + sl) * 32;
-  if (blockIdx.x * (GV_WARPS / KS) * 32 >= a.H) return;  // whole CTA out of range (uniform)
-  const bool rows_ok = row0 < a.H;  // H is a multiple of 128, so then all 32 rows are
+  const int sl = warp / KS, kq = warp % KS;  // slice set within the CTA, K part
+  const int row0 = (blockIdx.x * (GV_WARPS / KS) + sl) * 16 * RS;
+  if (blockIdx.x * (GV_WARPS / KS) * 16 * RS >= a.H) return;  // whole CTA out of range (uniform)
+  const bool rows_ok = row0 < a.H;  // H is a multiple of 128, a multiple of 16 * RS: then all 64 rows are
   const uint8_t *rec = expert_record(a, e);
   if (!rec) return;
   const int I = a.I, KB = I / 2, G = I / GROUP;
@@ -269,19 +287,17 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
   for (int n0 = 0; n0 < cnt; n0 += 8) {
     const bool ok = n0 + g < cnt;
     const uint16_t *hr = a.h + int64_t(lo + (ok ? n0 + g : 0)) * I + t * 32;
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[RS][4] = {};
     const int ngrp = rows_ok && kq < G ? (G - 1 - kq) / KS + 1 : 0;
     uint4 *ring = rings[warp];
     auto issue = [&](int i) {
       const int grp = kq + i * KS;
-      uint4 *d = ring + (i % GV_DEPTH_DOWN) * (4 * 32) + lane;
-      cp_async16(d, dq0 + grp * 64);
-      cp_async16(d + 32, dq0 + 8 * KB + grp * 64);
-      cp_async16(d + 64, dq0 + 16 * KB + grp * 64);
-      cp_async16(d + 96, dq0 + 24 * KB + grp * 64);
+      uint4 *d = ring + (i % DEPTH) * (NP * 32) + lane;
+#pragma unroll
+      for (int j = 0; j < NP; ++j) cp_async16(d + 32 * j, dq0 + j * 8 * KB + grp * 64);
     };
 #pragma unroll
-    for (int i = 0; i < GV_DEPTH_DOWN - 1; ++i) {
+    for (int i = 0; i < DEPTH - 1; ++i) {
       if (i < ngrp) issue(i);
       cp_async_commit();
     }
@@ -289,46 +305,57 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       xn[q] = ok && ngrp > 0 ? *(reinterpret_cast<const uint4 *>(hr + kq * GROUP) + q) : make_uint4(0, 0, 0, 0);
-    uint16_t s00 = 0, s01 = 0, s10 = 0, s11 = 0;  // scales of rows g, g+8 (slice 0) and g+16, g+24 (slice 1)
-    if (ngrp > 0) { s00 = ds[kq]; s01 = ds[8 * G + kq]; s10 = ds[16 * G + kq]; s11 = ds[24 * G + kq]; }
+    uint32_t sn[RS];  // BF16 scale pairs of rows (g + 16 s, g + 16 s + 8)
+    auto load_s = [&](int grp) {
+#pragma unroll
+      for (int r = 0; r < RS; ++r)
+        sn[r] = uint32_t(ds[16 * r * G + grp]) | (uint32_t(ds[(16 * r + 8) * G + grp]) << 16);
+    };
+    if (ngrp > 0) load_s(kq);
     for (int i = 0; i < ngrp; ++i) {
       const int grp = kq + i * KS;
-      if (i + GV_DEPTH_DOWN - 1 < ngrp) issue(i + GV_DEPTH_DOWN - 1);
+      if (i + DEPTH - 1 < ngrp) issue(i + DEPTH - 1);
       cp_async_commit();
       uint4 xb[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) xb[q] = xn[q];
-      const float c00 = bf16_to_f(s00), c01 = bf16_to_f(s01), c10 = bf16_to_f(s10), c11 = bf16_to_f(s11);
+      uint32_t sc[RS];
+#pragma unroll
+      for (int r = 0; r < RS; ++r) sc[r] = sn[r];
       if (i + 1 < ngrp) {
-        s00 = ds[grp + KS]; s01 = ds[8 * G + grp + KS]; s10 = ds[16 * G + grp + KS]; s11 = ds[24 * G + grp + KS];
+        load_s(grp + KS);
         if (ok) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) xn[q] = *(reinterpret_cast<const uint4 *>(hr + (grp + KS) * GROUP) + q);
         }
       }
-      cp_async_wait<GV_DEPTH_DOWN - 1>();  // group i's copies (this lane's) have landed
-      const uint4 *sr = ring + (i % GV_DEPTH_DOWN) * (4 * 32) + lane;
-      const uint4 w0 = sr[0], w1 = sr[32], w2 = sr[64], w3 = sr[96];
-      float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_group(p0, w0, w1, xb);
-      mma_group(p1, w2, w3, xb);
-      a0[0] = fmaf(c00, p0[0], a0[0]); a0[1] = fmaf(c00, p0[1], a0[1]);
-      a0[2] = fmaf(c01, p0[2], a0[2]); a0[3] = fmaf(c01, p0[3], a0[3]);
-      a1[0] = fmaf(c10, p1[0], a1[0]); a1[1] = fmaf(c10, p1[1], a1[1]);
-      a1[2] = fmaf(c11, p1[2], a1[2]); a1[3] = fmaf(c11, p1[3], a1[3]);
+      cp_async_wait<DEPTH - 1>();  // group i's copies (this lane's) have landed
+      const uint4 *sr = ring + (i % DEPTH) * (NP * 32) + lane;
+#pragma unroll
+      for (int r = 0; r < RS; ++r) {
+        float p[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_group(p, sr[64 * r], sr[64 * r + 32], xb);
+        const float c0 = bf16_lo(sc[r]), c1 = bf16_hi(sc[r]);
+        acc[r][0] = fmaf(c0, p[0], acc[r][0]); acc[r][1] = fmaf(c0, p[1], acc[r][1]);
+        acc[r][2] = fmaf(c1, p[2], acc[r][2]); acc[r][3] = fmaf(c1, p[3], acc[r][3]);
+      }
     }
-    if (KS > 1) {  // K parts 1.. hand their sums to part 0 of the slice pair
+    if (KS > 1) {  // K parts 1.. hand their sums to part 0 of the slice set
       __syncthreads();
       if (kq > 0) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) { red[kq - 1][sl][c][lane] = a0[c]; red[kq - 1][sl][4 + c][lane] = a1[c]; }
+        for (int r = 0; r < RS; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) red[kq - 1][sl][4 * r + c][lane] = acc[r][c];
       }
       __syncthreads();
       if (kq == 0) {
 #pragma unroll
         for (int q = 0; q < KS - 1; ++q)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) { a0[c] += red[q][sl][c][lane]; a1[c] += red[q][sl][4 + c][lane]; }
+          for (int r = 0; r < RS; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[r][c] += red[q][sl][4 * r + c][lane];
       }
     }
     // accumulator (c0, c1) = row g, tokens 2t, 2t+1; (c2, c3) = row g+8
@@ -337,10 +364,11 @@ __global__ void __launch_bounds__(GV_WARPS * 32) gemv_down_kernel(const FfnArgs 
       const int r = n0 + 2 * t + c;
       if (kq == 0 && rows_ok && r < cnt) {
         float *yr = a.y + int64_t(lo + r) * a.H + row0 + g;
-        yr[0] = a0[c];
-        yr[8] = a0[2 + c];
-        yr[16] = a1[c];
-        yr[24] = a1[2 + c];
+#pragma unroll
+        for (int s = 0; s < RS; ++s) {
+          yr[16 * s] = acc[s][c];
+          yr[16 * s + 8] = acc[s][2 + c];
+        }
       }
     }
   }
@@ -353,7 +381,7 @@ static cudaError_t launch_gemv_pair(const FfnArgs &a, cudaStream_t s) {
   cudaError_t e = launch_pdl(gemv_gateup_kernel<KS>, g1, dim3(GV_WARPS * 32), 0, s, a);
   if (e != cudaSuccess) return e;
   count_launches(1);
-  dim3 g2((a.H + rows_per_cta * 2 - 1) / (rows_per_cta * 2), a.E);  // two slices per warp
+  dim3 g2((a.H + rows_per_cta * DOWN_RS - 1) / (rows_per_cta * DOWN_RS), a.E);  // DOWN_RS slices per warp
   e = launch_pdl(gemv_down_kernel<KS>, g2, dim3(GV_WARPS * 32), 0, s, a);
   if (e == cudaSuccess) count_launches(1);
   return e;
@@ -395,7 +423,7 @@ int launch_ffn_sequential(const FfnArgs &a, cudaStream_t s) {
                    dim3(GV_WARPS * 32), 0, s, b);
     if (err == cudaSuccess) {
       count_launches(1);
-      err = launch_pdl(gemv_down_kernel<KS>, dim3((a.H + rows_per_cta * 2 - 1) / (rows_per_cta * 2), 1),
+      err = launch_pdl(gemv_down_kernel<KS>, dim3((a.H + rows_per_cta * DOWN_RS - 1) / (rows_per_cta * DOWN_RS), 1),
                        dim3(GV_WARPS * 32), 0, s, b);
     }
     if (err != cudaSuccess)

@@ -61,12 +61,10 @@
 // of overlapped. Every wait is bounded (about two
 // seconds of %globaltimer); a wait that runs out flags MOE_DEVERR_TIMEOUT and
 // all roles drain and exit.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
 #include "ffn.cuh"
+#include "tma.cuh"
 
 namespace moe {
 namespace tc {
@@ -84,7 +82,6 @@ constexpr int TMA_B_WARP = 18;
 constexpr int WAITER_WARP = 19;
 constexpr int THREADS = 640;
 constexpr int HANDOFF_BAR = 1;  // named barrier: waiter warp + MMA warp
-constexpr uint64_t WAIT_NS = 2000000000ull;
 
 template <bool GATEUP>
 struct Cfg {
@@ -113,57 +110,8 @@ struct Cfg {
 };
 
 // ------------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
-}
-// TMA tile loads (no multicast): completion counted in bytes on `bar`.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, int c0, int c1, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, int c0, int c1, int c2, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-      : "memory");
-}
-// One lane of a converged warp (the lowest), chosen by elect.sync: the
-// issue idiom for tcgen05 and TMA instructions, whose operands then stay in
-// uniform registers.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t pred = 0;
-  asm volatile(
-      "{\n .reg .b32 r;\n .reg .pred p;\n elect.sync r|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(pred));
-  return pred != 0;
-}
+using namespace tma;
+
 // Named-barrier handoff between the waiter and the MMA warp (64 threads):
 // returns the number of participating threads whose predicate is true.
 __device__ __forceinline__ uint32_t handoff(uint32_t pred) {
@@ -174,7 +122,6 @@ __device__ __forceinline__ uint32_t handoff(uint32_t pred) {
                : "memory");
   return cnt;
 }
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -242,29 +189,10 @@ struct Shared {
 };
 constexpr int ROWEXP_SLOTS = 4;  // tiles in flight between the two: at most three
 
-// Bounded wait: false (and the CTA-wide abort flag set) after WAIT_NS, or
-// as soon as another role aborted unless `drain` is set (a drain wait only
-// gives up on its own time limit, so tensor memory is never released under
-// MMAs still in flight).
-__device__ __noinline__ bool wait_bounded(Shared &sh, uint64_t *bar, uint32_t parity, int32_t *err,
-                                          bool drain = false) {
-  // %globaltimer is read only every 256 polls (the first time after 256): a
-  // wait that ends soon never pays for the timer read.
-  uint64_t t0 = 0;
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try(bar, parity)) return true;
-    if ((spin & 255) == 0) {
-      if (!drain && *(volatile int32_t *)&sh.abort) return false;
-      const uint64_t now = globaltimer();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > WAIT_NS) {
-        atomicExch(&sh.abort, 1);
-        flag_error(err, MOE_DEVERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
+// Bounded wait on the CTA's abort flag (see tma::wait_bounded).
+__device__ __forceinline__ bool wait_bounded(Shared &sh, uint64_t *bar, uint32_t parity, int32_t *err,
+                                             bool drain = false) {
+  return tma::wait_bounded(&sh.abort, bar, parity, err, drain);
 }
 
 struct Tile {
@@ -632,7 +560,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace tc
 
-static int sm_count() {
+int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -647,7 +575,7 @@ static int sm_count() {
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against the driver library).
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   std::call_once(once, [] {
@@ -667,7 +595,7 @@ static bool map_rows_f16(CUtensorMap *m, const void *base, int rows, int cols) {
   const cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
   const cuuint32_t box[2] = {tc::BK, tc::BN};
   const cuuint32_t estr[2] = {1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -679,7 +607,7 @@ static bool map_codes(CUtensorMap *m, const uint8_t *bank, int64_t off, int64_t 
   const cuuint64_t strides[2] = {cuuint64_t(kd / 2), cuuint64_t(rec)};
   const cuuint32_t box[3] = {tc::BK / 2, tc::BM, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(bank + off), dims, strides, box, estr,
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(bank + off), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -694,7 +622,7 @@ int launch_ffn_tc(const FfnArgs &a, cudaStream_t s) {
                      minor);
   if (a.H % tc::BM || a.I % tc::BM)
     return set_error(MOE_ERR_UNSUPPORTED, "moe_grouped_w4a16_ffn: tensor-core path needs H, I multiples of 128");
-  if (!encode_fn())
+  if (!tensor_map_encoder())
     return set_error(MOE_ERR_UNSUPPORTED, "moe_grouped_w4a16_ffn: cuTensorMapEncodeTiled is not available");
   const int P = a.T * a.k;
   CUtensorMap tm_xs, tm_h, tm_gq, tm_uq, tm_dq;
