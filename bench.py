@@ -18,6 +18,10 @@ cpu_baseline: the CPU oracle (plain C, fp64, OpenMP over experts and tokens)
         on a bounded sample of the workload: whole passes of layer 0 at the
         bench's T, repeated for about ten seconds.
 
+The line also carries the rest of the decode sweep (T = 1, 4, 64), prefill
+entries (tensor-core path, against the BF16 peak), the sequential-W4 and BF16
+reference paths at T = 16, and slot-cache decode from a pinned host pool.
+
 --impl reference runs that oracle as the reference arm (rank 0 only).
 Multi-GPU: replicas only (each rank runs the whole workload on its own GPU;
 the layer has no exchange step), timed as the max over ranks.
@@ -67,6 +71,8 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true", help="leave the prefill entries out of the default line")
     ap.add_argument("--no-references", action="store_true",
                     help="leave the sequential-W4 and BF16 reference paths out of the default line")
+    ap.add_argument("--no-slotcache", action="store_true",
+                    help="leave the slot-cache decode entry out of the default line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tc", "seq"])
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "slotcache"],
@@ -420,6 +426,10 @@ def main():
         for shape, Tp in PREFILL_CASES:
             prefill[f"{shape}-T{Tp}"] = prefill_entry(a, shape, Tp, rank, world, P)
             torch.cuda.empty_cache()
+    slot = {}
+    if not a.no_slotcache:
+        slot = slotcache_entry(a)
+        torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         v, cores, desc = oracle_sample(a.T, seconds=10.0)
@@ -446,13 +456,14 @@ def main():
                                      else None),
                          "traffic_source": "ncu capture, scaled by active experts",
                          "peak_source": P["source"], "bytes_per_call": head["ffn_bytes_per_call"],
-                         "ms_per_call": head["ffn_ms_per_call"]},
+                         "ms_per_call": head["ffn_ms_per_call"], "n_active_mean": head["n_active_mean"]},
             "cpu_baseline": cpu,
             "gpu_launches": head["launches_per_step"] * a.steps,
             "clocks": head["clocks"],
             "sweep": sweep,
             "prefill": prefill,
             "references": refs,
+            "slotcache": slot,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -465,24 +476,24 @@ def main():
 PAGES_HIT_RATE = {8: 0.388, 16: 0.563, 32: 0.814, 64: None}
 
 
-def main_slotcache(a, rank, world, P):
+def slotcache_runs(layers, runs, steps, warmup):
     """Decode with every expert in pinned host memory and S GPU slots per
-    layer, for each S of --slots (a comma list; the pages' Table 1 sweeps 8,
-    16, 32 and 64 = all experts). T tokens per step (default 1), each an
-    independent routing stream that keeps each expert of its previous step
-    with probability 0.5. Per layer and step: route (weights of the drawn
-    ids), plan the step's experts in cache-sized waves, and per wave: host LRU
-    lookup, H2D fill of the misses on a side stream, grouped FFN through the
-    slot table (that wave's experts only), release; then the combine."""
+    layer, for each (T, S) of `runs` (the pages' Table 1 sweeps S = 8, 16, 32
+    and 64 = all experts). T tokens per step, each an independent routing
+    stream that keeps each expert of its previous step with probability 0.5.
+    Per layer and step: route (weights of the drawn ids), plan the step's
+    experts in cache-sized waves, and per wave: host LRU lookup, H2D fill of
+    the misses on a side stream, grouped FFN through the slot table (that
+    wave's experts only), release; then the combine. Returns the per-run
+    results, the pinned host -> device copy bandwidth measured in the same
+    run, and the pool's size."""
     import numpy as np
     import torch
 
     import synth
     M = __import__("w4a16_mixture_experts_moe_b200")
     from w4a16_mixture_experts_moe_b200.layer import LayerBuffers
-    L, T = a.layers, a.T if a.T != 16 else 1
-    slot_counts = [int(v) for v in str(a.slots).split(",")]
-    steps = a.steps if a.steps >= 16 else 128
+    L = layers
     stack = Stack(L, "auto")
     rec = stack.banks[0].rec
     pool = torch.empty(L * E * rec, dtype=torch.uint8, pin_memory=True)
@@ -490,14 +501,7 @@ def main_slotcache(a, rank, world, P):
         pool[l * E * rec:(l + 1) * E * rec].copy_(stack.banks[l].buf)
     stack.banks = None                       # the experts now live only in the pinned pool
     torch.cuda.empty_cache()
-    n_steps = a.warmup + steps
-    # routing[l][s] = ids [T][K] of step s in layer l
-    routing = [np.stack([synth.drawn_routing(l, E, K, n_steps, stream=t) for t in range(T)], axis=1)
-               for l in range(L)]
-    ids_dev = torch.from_numpy(np.stack(routing, axis=1).astype(np.int32)).cuda()   # [step][layer][T][K]
-    x0 = synth.activations(n_steps * T, H, device="cuda").view(n_steps, T, H)
-    bufs = [LayerBuffers(T, K, E, H, I) for _ in range(L)]
-    xs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    n_steps = warmup + steps
     side = torch.cuda.Stream()
     comp = torch.cuda.current_stream()
 
@@ -515,7 +519,14 @@ def main_slotcache(a, rank, world, P):
     pinned_gbs = probe_n * rec / (ev0.elapsed_time(ev1) / 1e3) / 1e9
     del dst
 
-    def run(S):
+    def run(T, S):
+        # routing[l][s] = ids [T][K] of step s in layer l
+        routing = [np.stack([synth.drawn_routing(l, E, K, n_steps, stream=t) for t in range(T)], axis=1)
+                   for l in range(L)]
+        ids_dev = torch.from_numpy(np.stack(routing, axis=1).astype(np.int32)).cuda()   # [step][layer][T][K]
+        x0 = synth.activations(n_steps * T, H, device="cuda").view(n_steps, T, H)
+        bufs = [LayerBuffers(T, K, E, H, I) for _ in range(L)]
+        xs = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
         slots = torch.empty(L * S * rec, dtype=torch.uint8, device="cuda")
         table = torch.full((L, E), -1, dtype=torch.int32, device="cuda")
         cache = M.SlotCache(L, E, S, rec, pool, slots, table)
@@ -544,7 +555,7 @@ def main_slotcache(a, rank, world, P):
                 cur = out
             return cur
 
-        for si in range(a.warmup):
+        for si in range(warmup):
             step(si)
         torch.cuda.synchronize()
         st0 = cache.stats()
@@ -553,7 +564,7 @@ def main_slotcache(a, rank, world, P):
         launches0 = M.moe_launch_counter()
         with ClockSampler(torch.cuda.current_device()) as clk:
             s0.record()
-            for si in range(a.warmup, n_steps):
+            for si in range(warmup, n_steps):
                 step(si)
             s1.record()
             torch.cuda.synchronize()
@@ -565,16 +576,27 @@ def main_slotcache(a, rank, world, P):
         err = sorted(set(M.moe_read_device_error(b.ffn_ws) for b in bufs))
         cache.close()
         del slots, table
-        return {"slots": S, "value": T * L / (ms / 1e3), "unit": "layer-tokens/s", "ms_per_step": ms,
+        return {"T": T, "slots": S, "value": T * L / (ms / 1e3), "unit": "layer-tokens/s", "ms_per_step": ms,
                 "decode_tokens_per_s": T * 1e3 / ms,
                 "hit_rate": None if S >= E else hits / max(1, hits + misses),
-                "pages_hit_rate_l4": PAGES_HIT_RATE.get(S),
+                "pages_hit_rate_l4": PAGES_HIT_RATE.get(S) if T == 1 else None,
                 "h2d_gb": h2d / 1e9, "h2d_gb_per_step": h2d / 1e9 / steps,
                 "h2d_achieved_gbs": h2d / (ms * steps / 1e3) / 1e9,
                 "waves_per_layer_step": n_waves[0] / (steps * L), "device_errors": err,
                 "gpu_launches": launches, "clocks": clk.summary()}
 
-    results = [run(S) for S in slot_counts]
+    results = [run(T, S) for T, S in runs]
+    del stack
+    return results, pinned_gbs, L * E * rec
+
+
+def main_slotcache(a, rank, world, P):
+    """The slot-cache decode workload on its own line (--workload slotcache):
+    T = --T (1 unless given), one run per slot count of --slots."""
+    L, T = a.layers, a.T if a.T != 16 else 1
+    slot_counts = [int(v) for v in str(a.slots).split(",")]
+    steps = a.steps if a.steps >= 16 else 128
+    results, pinned_gbs, pool_bytes = slotcache_runs(L, [(T, S) for S in slot_counts], steps, a.warmup)
     head = next((r for r in results if r["slots"] == 16), results[0])
     if rank == 0:
         line = {
@@ -584,13 +606,26 @@ def main_slotcache(a, rank, world, P):
             "config": {"workload": f"olmoe-{L}L-slotcache-decode", "T": T, "layers": L,
                        "slots_per_layer": head["slots"], "H": H, "I": I, "E": E, "k": K,
                        "routing": "drawn per token stream, keep-probability 0.5",
-                       "pool": f"{L * E * rec / 1e9:.2f} GB pinned host", "parallelism": f"replicas{world}"},
+                       "pool": f"{pool_bytes / 1e9:.2f} GB pinned host", "parallelism": f"replicas{world}"},
             "decode_tokens_per_s": head["decode_tokens_per_s"], "hit_rate": head["hit_rate"],
             "h2d_gb": head["h2d_gb"], "h2d_achieved_gbs": head["h2d_achieved_gbs"], "pinned_copy_gbs": pinned_gbs,
             "device_errors": head["device_errors"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
             "slot_sweep": {str(r["slots"]): r for r in results},
         }
         print(json.dumps(line), flush=True)
+
+
+def slotcache_entry(a):
+    """The slot-cache entry of the default line: the 16-layer stack decoding
+    from the pinned pool at T = 1 for 8, 16, 32 and 64 slots per layer, and
+    at T = 4 through 16 slots (about 27 distinct experts a step: two waves)."""
+    runs = [(1, 8), (1, 16), (1, 32), (1, 64), (4, 16)]
+    results, pinned_gbs, pool_bytes = slotcache_runs(LAYERS, runs, 48, 4)
+    out = {"pool_gb_pinned_host": pool_bytes / 1e9, "pinned_copy_gbs": pinned_gbs, "steps": 48,
+           "routing": "drawn per token stream, keep-probability 0.5"}
+    for r in results:
+        out[f"T{r['T']}-S{r['slots']}"] = r
+    return out
 
 
 # The pages' own ratios for these two comparisons, measured on one L4 on the
