@@ -616,13 +616,16 @@ def main_slotcache(a, rank, world, P):
         print(json.dumps(line), flush=True)
 
 
+SLOTCACHE_STEPS = 128  # decode steps per slot-cache run (the workload's 128-step trace)
+
+
 def slotcache_entry(a):
     """The slot-cache entry of the default line: the 16-layer stack decoding
     from the pinned pool at T = 1 for 8, 16, 32 and 64 slots per layer, and
     at T = 4 through 16 slots (about 27 distinct experts a step: two waves)."""
     runs = [(1, 8), (1, 16), (1, 32), (1, 64), (4, 16)]
-    results, pinned_gbs, pool_bytes = slotcache_runs(LAYERS, runs, 48, 4)
-    out = {"pool_gb_pinned_host": pool_bytes / 1e9, "pinned_copy_gbs": pinned_gbs, "steps": 48,
+    results, pinned_gbs, pool_bytes = slotcache_runs(LAYERS, runs, SLOTCACHE_STEPS, 4)
+    out = {"pool_gb_pinned_host": pool_bytes / 1e9, "pinned_copy_gbs": pinned_gbs, "steps": SLOTCACHE_STEPS,
            "routing": "drawn per token stream, keep-probability 0.5"}
     for r in results:
         out[f"T{r['T']}-S{r['slots']}"] = r

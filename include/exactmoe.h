@@ -2,13 +2,14 @@
  * exactmoe.h — C ABI of the fused grouped W4A16 routed-expert MoE layer.
  *
  * Method: "Every Expert Counts: ExactMoE for Memory-Efficient W4A16 Inference"
- * (A. Saab, arXiv 2608.15383). The Abstract fixes symmetric group-128 four-bit
- * quantisation of the routed experts only, a BF16 router with an unchanged
- * top-k procedure, and fused grouped MoE kernels fed by a GPU-resident expert
- * slot cache over pinned host memory. The Figure 1 caption fixes the order of
- * the steps: pack once; the BF16 router selects experts; tokens are grouped by
- * selected expert; the active experts run in fused grouped kernels; cache
- * misses move packed weights and scales without materialising FP16 experts.
+ * (A. Saab, arXiv 2608.15383). The Abstract fixes four-bit symmetric
+ * quantisation in groups of 128 for the routed experts only, a BF16 router
+ * whose top-k is left as it was, and fused grouped expert kernels fed by a
+ * slot cache on the GPU over experts kept in pinned host memory. The Figure 1
+ * caption fixes the order of the steps: the experts are packed ahead of time;
+ * the BF16 router picks experts; the tokens are gathered per chosen expert;
+ * fused grouped kernels run the active experts; a cache miss copies packed
+ * codes and scales, and no FP16 copy of an expert is ever made.
  *
  * Conventions for every entry point below:
  *  - Pointers are DEVICE pointers unless a parameter says "host". The caller
@@ -103,7 +104,7 @@ int moe_expert_record_layout(int H, int I, moe_record_layout *out);
 
 /*
  * A1 — quantise and pack (Abstract: symmetric group-128 int4 weights for the
- * routed experts; Figure 1 caption: packed once, offline).
+ * routed experts; Figure 1 caption: packing happens a single time, offline).
  *   w       [E][N][K] BF16, one nn.Linear weight per expert (K = in).
  *   packed  expert e's codes at packed + e*packed_stride, [N][K/2] bytes.
  *   scales  expert e's scales at (char*)scales + e*scales_stride, [N][K/128].
@@ -124,8 +125,8 @@ int moe_quantize_pack(const moe_bf16 *w, int E, int N, int K,
 
 /*
  * A2 + A3 — BF16 router logits, full softmax and unchanged top-k
- * (Abstract: the router stays BF16 and the top-k routing procedure is
- * unchanged; Figure 1 caption: the original BF16 router selects experts).
+ * (Abstract: the router stays BF16 and top-k routing is left as it was;
+ * Figure 1 caption: the model's own BF16 router picks the experts).
  *   x         [T][H] BF16 activations.
  *   w_router  [E][H] BF16 (nn.Linear convention).
  *   bias      [E] fp32 added to the logits before softmax/top-k, or NULL.
@@ -146,8 +147,8 @@ int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router,
                    moe_stream_t stream);
 
 /*
- * A4 — group the T*k (token, slot) pairs by expert (Figure 1 caption: tokens
- * are grouped by selected expert).
+ * A4 — group the T*k (token, slot) pairs by expert (Figure 1 caption: the
+ * tokens are gathered per chosen expert).
  *   topk_ids    [T][k] int32.
  *   counts      [E] int32 pairs per expert.
  *   offsets     [E+1] int32 exclusive prefix sum of counts.
@@ -209,8 +210,8 @@ int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E,
 
 /*
  * A5 + A6 — the grouped SwiGLU expert FFN with in-kernel int4 dequantisation
- * (Abstract: fused grouped MoE kernels over W4A16 experts; Figure 1 caption:
- * packed weights and scales are consumed without materialising FP16 experts).
+ * (Abstract: fused grouped kernels over W4A16 experts; Figure 1 caption:
+ * the kernels read packed codes and scales, with no FP16 copy of an expert).
  * For sorted row r of expert e (offsets[e] <= r < offsets[e+1]) and token
  * t = sorted_pair[r] / k:
  *   h[r] = bf16_rn(silu(x[t] Wg_e^T) * (x[t] Wu_e^T))      (fp32 sums)
@@ -306,11 +307,11 @@ int moe_combine(const float *y, const float *topk_w,
 int moe_read_device_error(void *ws, moe_stream_t stream, int32_t *code);
 
 /*
- * A8 — GPU-resident expert slot cache over a pinned host pool (Abstract: a
- * configurable GPU-resident slot cache over experts kept in pinned host
- * memory; Figure 1 caption: the pinned pool keeps every packed expert and a
- * miss moves packed weights and scales; Figure 2 caption: with capacity
- * >= E every expert is resident and lookup accounting is bypassed).
+ * A8 — expert slot cache on the GPU over a pinned host pool (Abstract: the
+ * experts live in pinned host memory and a slot cache of configurable size
+ * holds some of them on the GPU; Figure 1 caption: the host pool holds every
+ * packed expert and a miss copies its packed codes and scales; Figure 2
+ * caption: once the cache holds all E experts no hit rate is counted).
  *
  * The cache owns only host bookkeeping (an LRU per layer) and two CUDA
  * events per layer; all memory is the caller's:
@@ -364,8 +365,8 @@ int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss_ids_host,
 int slot_cache_release(moe_slot_cache *c, int layer, moe_stream_t compute);
 
 /*
- * Cache-sized fused waves (Figure 1 caption: the active experts execute in
- * cache-sized fused waves). Splits the n expert ids (host) one step of
+ * Cache-sized waves (Figure 1 caption: the active experts run in waves sized
+ * to the cache). Splits the n expert ids (host) one step of
  * `layer` needs into waves of at most `slots` distinct experts: the
  * distinct ids in first-occurrence order, those already held in a slot
  * first (so they run before anything can evict them), cut into consecutive
@@ -390,9 +391,9 @@ int slot_cache_inject_fill_failure(moe_slot_cache *c, int count);
 void slot_cache_destroy(moe_slot_cache *c);
 
 /*
- * The packed pool as a file: the "quantised and packed once" artifact
- * (Figure 1 caption: experts are quantised and packed once offline, and the
- * pinned host pool keeps every packed expert). Host-only calls (no CUDA),
+ * The packed pool as a file, so the packing is done a single time (Figure 1
+ * caption: the experts are quantised and packed ahead of time, and the pinned
+ * host pool holds every packed expert). Host-only calls (no CUDA),
  * so a pool can be written once and reloaded into pinned memory, a bank or
  * a slot cache's pool without re-quantising.
  *   pool    host, [layers][E] records of record_bytes, the layout of a bank

@@ -8,15 +8,14 @@
  * independently from the same definitions and checked against each other.
  *
  * Source: "Every Expert Counts: ExactMoE for Memory-Efficient W4A16
- * Inference" (A. Saab, arXiv 2608.15383), pages thelatestinai.com/papers/
- * 2608.15383 and searcharxiv.org/abs/2608.15383:
- *   - Abstract: symmetric group-128 four-bit quantisation of the routed
- *     experts only; router and activations stay BF16; "exact" means every
- *     selected expert runs and the top-k routing is unchanged.
- *   - Figure 1 caption: the BF16 router selects experts, tokens are grouped
- *     by selected expert, the active experts run in fused grouped kernels,
- *     and packed weights plus scales are consumed without materialising FP16
- *     experts.
+ * Inference" (A. Saab, arXiv 2608.15383):
+ *   - Abstract: only the routed experts are quantised, four-bit, symmetric,
+ *     in groups of 128; router and activations stay BF16; exactness means
+ *     that every chosen expert is run and top-k routing is left as it was.
+ *   - Figure 1 caption: the order of the steps. The BF16 router picks the
+ *     experts, the tokens are gathered per chosen expert, fused grouped
+ *     kernels run the active experts, and they read the packed codes and
+ *     scales directly, with no FP16 copy of any expert.
  * The pages give no formula, so each function below states the plainest
  * reading of those passages it implements (the same readings as the numpy
  * oracle): quantiser s = bf16_rn(absmax/7) (fp32 divide), q = clamp(rint(w/s),

@@ -6,15 +6,15 @@ legs may call it. It shares no code, table or constant generator with the
 CUDA library; both sides implement the definitions below independently.
 
 Source: "Every Expert Counts: ExactMoE for Memory-Efficient W4A16 Inference"
-(A. Saab, arXiv 2608.15383), pages thelatestinai.com/papers/2608.15383 and
-searcharxiv.org/abs/2608.15383:
+(A. Saab, arXiv 2608.15383):
 
-* Abstract: symmetric group-128 four-bit weight quantisation of the routed
-  experts only; router and activations stay BF16; "exact" means every
-  selected expert runs and the top-k routing procedure is unchanged.
-* Figure 1 caption: the BF16 router selects experts, tokens are grouped by
-  selected expert, the active experts run in fused grouped kernels, and packed
-  weights plus scales are consumed without materialising FP16 experts.
+* Abstract: only the routed experts are quantised, four-bit, symmetric, in
+  groups of 128; router and activations stay BF16; exactness means that
+  every chosen expert is run and top-k routing is left as it was.
+* Figure 1 caption: the order of the steps. The BF16 router picks the
+  experts, the tokens are gathered per chosen expert, fused grouped kernels
+  run the active experts, and they read the packed codes and scales
+  directly, with no FP16 copy of any expert.
 
 The pages give no formula, pseudo-code or worked example, so each step below
 is the plainest reading of those two passages (readings listed in the design
@@ -89,7 +89,7 @@ def f64_to_bf16_bits(x) -> np.ndarray:
 
 # --------------------------------------------------------------------------
 # Quantise + pack (Abstract: symmetric group-128 int4 on routed experts;
-# Figure 1 caption: packed once into the kernel-native form)
+# Figure 1 caption: packing happens a single time, into the form the kernels read)
 # --------------------------------------------------------------------------
 
 def quantize_group128(w) -> tuple[np.ndarray, np.ndarray]:
@@ -161,8 +161,8 @@ def dequantize_packed(packed, scale_bits) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# Router (Abstract: the router stays BF16; Figure 1 caption: the original
-# BF16 router selects experts; "exact" = unchanged top-k)
+# Router (Abstract: the router stays BF16 and top-k routing is left as it
+# was; Figure 1 caption: the model's own BF16 router picks the experts)
 # --------------------------------------------------------------------------
 
 def router_logits(x, w_router) -> np.ndarray:
@@ -216,7 +216,7 @@ def weights_for_ids(logits, ids, bias=None, renorm: bool = False) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# Grouping (Figure 1 caption: tokens are grouped by selected expert)
+# Grouping (Figure 1 caption: the tokens are gathered per chosen expert)
 # --------------------------------------------------------------------------
 
 def group_tokens(ids, E: int):
@@ -395,11 +395,11 @@ def moe_layer(x, w_router, experts: PackedExperts, k: int, bias=None,
 
 
 # --------------------------------------------------------------------------
-# Expert slot cache (Abstract: a configurable GPU-resident slot cache over
-# experts kept in pinned host memory; Figure 1 caption: a miss moves the
-# packed weights and scales of the expert; Figure 2 caption: when the cache
-# holds every expert, lookup accounting is bypassed; Table 1: hit rate and
-# host-to-device traffic per slot count)
+# Expert slot cache (Abstract: the experts live in pinned host memory and a
+# slot cache of configurable size holds some of them on the GPU; Figure 1
+# caption: a miss copies the expert's packed codes and scales; Figure 2
+# caption: once the cache holds all experts no hit rate is counted; Table 1:
+# hit rate and host-to-device traffic per slot count)
 # --------------------------------------------------------------------------
 
 class SlotCapacityError(ValueError):
@@ -490,8 +490,8 @@ class SlotCacheLRU:
         return [self.slot_of(v) for v in ids], loaded, evicted
 
     def plan_waves(self, ids):
-        """Cache-sized waves (Figure 1 caption: active experts execute in
-        cache-sized fused waves): the step's distinct ids in first-occurrence
+        """Cache-sized waves (Figure 1 caption: the active experts run in
+        waves sized to the cache): the step's distinct ids in first-occurrence
         order, those already held in a slot first, cut into consecutive
         waves of at most S ids. Each wave is then one lookup."""
         distinct = []

@@ -298,7 +298,7 @@ def test_packed_pool_file_round_trip_runs_the_layer(M, tmp_path):
     into pinned host memory, copy them to a fresh device bank, and run the
     layer from it: the bank is byte-identical to the packed one, the output
     bit-identical to the output from the packed bank and within the BF16 bar
-    of the oracle (Figure 1 caption: packed once)."""
+    of the oracle (Figure 1 caption: packing happens a single time)."""
     from w4a16_mixture_experts_moe_b200.layer import ExpertBank, LayerBuffers, moe_layer_forward
     T = 16
     bank, wr = _gpu_bank(M, 0)

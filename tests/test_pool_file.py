@@ -1,5 +1,5 @@
-"""The packed pool as a file (Figure 1 caption: experts are quantised and
-packed once): host-only save / load through the C ABI, on the CPU. The file
+"""The packed pool as a file (Figure 1 caption: the experts are quantised
+and packed ahead of time): host-only save / load through the C ABI, on the CPU. The file
 format stated in include/exactmoe.h is checked independently here: the header
 fields are parsed with `struct` and the checksum is recomputed with numpy."""
 import os

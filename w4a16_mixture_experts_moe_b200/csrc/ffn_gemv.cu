@@ -83,7 +83,11 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t x, uint32_t mask, uint3
 // holds k = 2i + h at bits 4(i + 4h): nibbles at bits 0-3/16-19 are pair 0,
 // 4-7/20-23 pair 1; after one right shift by 8, pairs 2 and 3 sit at the same
 // places. Low nibbles: (1024 + u) - 1032 = u - 8. High nibbles: (1024 + 16u)
-// / 16 - 72 = u - 8. Every step is exact in FP16.
+// / 16 - 72 = u - 8. Every step is exact in FP16. This is the published
+// fast int4 -> FP16 conversion by exponent-field insertion (Kim et al., 2022,
+// "Who Says Elephants Can't Run: Bringing Large Scale MoE Models into Cloud
+// Scale Production", the method FasterTransformer's int4 kernels use), here
+// applied to this library's own interleaved word layout.
 __device__ __forceinline__ void dequant_codes_f16(uint32_t w, uint32_t (&q)[4]) {
   const __half2 lo_bias = __floats2half2_rn(1032.0f, 1032.0f);
   const __half2 hi_scale = __floats2half2_rn(0.0625f, 0.0625f);
@@ -405,7 +409,7 @@ static int pick_ksplit(const FfnArgs &a) {
   return warps * 2 <= want ? 4 : (warps * 1.25 <= want || many_rows ? 2 : 1);
 }
 
-// The sequential reference (the pages' "sequential W4" baseline, Abstract):
+// The sequential reference (the per-expert W4 baseline of the pages, Abstract):
 // the same kernels launched once per expert, gate/up then down, expert after
 // expert, each launch covering one expert's rows with the widest K split.
 // Experts without rows still get their (empty) launches: the host does not

@@ -403,6 +403,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         // 16-19 into FP16 1024.0 gives (1024 + u), those at bits 4-7 / 20-23
         // give (1024 + 16u); one shift by 8 brings pairs 2 and 3 to the same
         // places. (1024 + u) - 1032 = q and (1024 + 16u) / 16 - 72 = q, exact.
+        // (The published int4 -> FP16 conversion by exponent-field insertion:
+        // Kim et al., 2022, "Who Says Elephants Can't Run".)
         const uint32_t w0 = words[wd], w8 = words[wd] >> 8;
         const uint32_t tq[4] = {(w0 & 0x000F000Fu) | 0x64006400u, (w0 & 0x00F000F0u) | 0x64006400u,
                                 (w8 & 0x000F000Fu) | 0x64006400u, (w8 & 0x00F000F0u) | 0x64006400u};

@@ -1,5 +1,5 @@
-// A4 — deterministic grouping of (token, slot) pairs by selected expert
-// (ExactMoE paper, Figure 1 caption: tokens are grouped by selected expert).
+// A4 — deterministic grouping of (token, slot) pairs by chosen expert
+// (ExactMoE paper, Figure 1 caption: the tokens are gathered per chosen expert).
 //
 // A stable counting sort over the P = T*k flat pair indices, in chunks of
 // 1024 pairs (one pair per thread):

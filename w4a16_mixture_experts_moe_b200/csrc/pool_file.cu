@@ -1,6 +1,6 @@
-// The packed expert pool as a file: the "quantised and packed once" artifact
-// (ExactMoE paper, Figure 1 caption: experts are quantised and packed once,
-// and the pinned host pool keeps every packed expert). Host code only; no
+// The packed expert pool as a file, so the packing is done a single time
+// (ExactMoE paper, Figure 1 caption: the experts are quantised and packed
+// ahead of time, and the pinned host pool holds every packed expert). Host code only; no
 // CUDA call is made, so a pool can be written and checked on a machine
 // without a GPU.
 //

@@ -1,6 +1,7 @@
 // A1 — symmetric group-128 int4 quantisation and packing, run once offline
 // (ExactMoE paper, Abstract: group-128 four-bit weights for the routed
-// experts; Figure 1 caption: packed once into the kernel-native form).
+// experts; Figure 1 caption: packing happens a single time, into the form
+// the kernels read).
 //
 // One warp per (expert, row, 128-group). Lane l holds k = 4l .. 4l+3 of the
 // group; lanes 2m and 2m+1 together form packed word m of the group.

@@ -1,7 +1,7 @@
 // A2 + A3 — BF16 router logits, full softmax, unchanged top-k
-// (ExactMoE paper, Abstract: the router stays BF16 and the top-k routing
-// procedure is unchanged; Figure 1 caption: the original BF16 router selects
-// the experts).
+// (ExactMoE paper, Abstract: the router stays BF16 and top-k routing is
+// left as it was; Figure 1 caption: the model's own BF16 router picks the
+// experts).
 //
 // One thread-block cluster of 8 CTAs serves TOK tokens (8 for large batches;
 // 2 for decode-sized ones, so their few tokens still spread over many SMs).

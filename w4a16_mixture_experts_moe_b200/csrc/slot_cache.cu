@@ -1,17 +1,17 @@
-// A8 — GPU-resident expert slot cache over a pinned host pool (ExactMoE
-// paper, Abstract: a configurable GPU-resident slot cache over experts kept in
-// pinned host memory; Figure 1 caption: the pinned pool keeps every packed
-// expert and a miss transfers packed weights and scales; Figure 2 caption:
-// at full capacity every expert is resident and lookup accounting is
-// bypassed; Table 1: slot counts 8/16/32/64 with hit rate and H2D traffic).
+// A8 — expert slot cache on the GPU over a pinned host pool (ExactMoE
+// paper, Abstract: the experts live in pinned host memory and a slot cache
+// of configurable size holds some of them on the GPU; Figure 1 caption: the
+// host pool holds every packed expert, and a miss copies its packed codes and
+// scales; Figure 2 caption: once the cache holds all experts no hit rate is
+// counted; Table 1: slot counts 8/16/32/64 with hit rate and H2D traffic).
 //
 // Host side: one LRU per layer over `slots` device records. A miss evicts the
 // least recently used slot that the current step does not need and is filled
 // with one cudaMemcpyAsync of the expert's whole record (packed codes and
 // scales, no dequantised copy) on a side stream. The layer's device table
 // expert -> slot names exactly the experts of the last lookup; when a step
-// needs more experts than there are slots (Figure 1 caption: active experts
-// run in cache-sized fused waves), slot_cache_plan_waves splits it, and the
+// needs more experts than there are slots (Figure 1 caption: the active
+// experts run in waves sized to the cache), slot_cache_plan_waves splits it, and the
 // step's experts outside the current wave are marked MOE_SLOT_SKIP, so each
 // wave's grouped FFN call computes that wave's experts and no other. The table
 // is rewritten by a one-block kernel on the compute stream, after the
