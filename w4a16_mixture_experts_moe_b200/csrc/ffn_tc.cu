@@ -163,6 +163,15 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 // after tcgen05.wait::ld, and a separate wait statement (tied to the loads
 // by nothing but a memory clobber) lets the compiler schedule arithmetic on
 // those registers ahead of it, reading whatever they held before.
+__device__ __forceinline__ void tmem_ld16(uint32_t ta, uint32_t (&a)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+        "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15])
+      : "r"(ta)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, uint32_t (&a)[16], uint32_t (&b)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n"
@@ -184,15 +193,18 @@ struct Shared {
   uint64_t tmem_full[2], tmem_empty[2], drain;
   uint32_t tmem_base;
   int32_t abort;
-  int32_t total_tiles;
+  int32_t total_tiles, full_tiles;
   int32_t off[MAX_E + 1];    // group offsets
-  int32_t tstart[MAX_E + 1]; // first tile of each expert
+  int32_t tstart[MAX_E + 1]; // first full-width tile of each expert (full tiles come first)
+  int16_t prow[MAX_E];       // rows of the expert's last, narrower token tile (0: none)
+  int16_t porder[MAX_E];     // experts with a narrower tile, widest first (ties: lower index)
   // power-of-two exponent of each weight row of a tile, written by the
   // dequant warps at the tile's start, read by the epilogue after the tile's
   // accumulator is complete; indexed by tile % ROWEXP_SLOTS ([block][row])
   int16_t row_exp[4][2][128];
 };
 constexpr int ROWEXP_SLOTS = 4;  // tiles in flight between the two: at most three
+static_assert(sizeof(Shared) <= 6144, "shared tables budget");
 
 // Bounded wait on the CTA's abort flag (see tma::wait_bounded).
 __device__ __forceinline__ bool wait_bounded(Shared &sh, uint64_t *bar, uint32_t parity, int32_t *err,
@@ -234,21 +246,43 @@ __device__ __forceinline__ int row_exponent(const uint16_t *srow, int G) {
   return -4 - e;
 }
 
+// The tile list, in the order it is handed out: every full-width (BN-token)
+// tile first, expert by expert, then each expert's narrower last token tile,
+// widest first. A narrow tile costs nearly the dequantisation and k-step
+// chain of a full one for a fraction of its MMAs, so handing the tiles out
+// from the longest down evens out the CTAs' finishing times (the
+// longest-processing-time-first rule).
 template <int FW>
 __device__ __forceinline__ Tile decode_tile(const Shared &sh, int E, int FT, int t) {
-  int lo_e = 0, hi_e = E;  // largest e with tstart[e] <= t
-  while (hi_e - lo_e > 1) {
-    const int mid = (lo_e + hi_e) >> 1;
-    if (sh.tstart[mid] <= t) lo_e = mid; else hi_e = mid;
-  }
   Tile x;
-  x.e = lo_e;
-  const int r = t - sh.tstart[lo_e];
-  x.lo = sh.off[lo_e];
-  x.n0 = (r / FT) * BN;
-  x.f0 = (r % FT) * FW;
-  x.nvalid = min(BN, sh.off[lo_e + 1] - x.lo - x.n0);
+  if (t < sh.full_tiles) {
+    int lo_e = 0, hi_e = E;  // largest e with tstart[e] <= t
+    while (hi_e - lo_e > 1) {
+      const int mid = (lo_e + hi_e) >> 1;
+      if (sh.tstart[mid] <= t) lo_e = mid; else hi_e = mid;
+    }
+    const int r = t - sh.tstart[lo_e];
+    x.e = lo_e;
+    x.n0 = (r / FT) * BN;
+    x.f0 = (r % FT) * FW;
+    x.nvalid = BN;
+  } else {
+    const int q = t - sh.full_tiles;
+    x.e = sh.porder[q / FT];
+    x.f0 = (q % FT) * FW;
+    x.nvalid = sh.prow[x.e];
+    x.n0 = sh.off[x.e + 1] - sh.off[x.e] - x.nvalid;
+  }
+  x.lo = sh.off[x.e];
   return x;
+}
+
+// The CTA's i-th tile: position i*G + b of the list on even rounds and
+// i*G + (G - 1 - b) on odd ones (a snake over the CTAs), so that the CTAs
+// which took the longest tiles of one round take the shortest of the next.
+__device__ __forceinline__ int sched_pos(int i) {
+  const int G = int(gridDim.x), b = int(blockIdx.x);
+  return i * G + ((i & 1) ? G - 1 - b : b);
 }
 
 // tm_b: activation rows in group order (gate/up: FP16 x gathered by the
@@ -294,7 +328,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (warp == 0) {  // per-expert tile counts -> prefix (experts without a slot get none)
-    int v[8], local = 0;
+    int v[8], local = 0, nparts = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane * 8 + i;
@@ -302,11 +336,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (e <= E) sh.off[e] = a.offsets[e];
       if (e < E) {
         const int cnt = a.offsets[e + 1] - a.offsets[e];
+        int rows = 0;
         if (cnt > 0) {
           const int slot = a.expert_slot ? a.expert_slot[e] : e;
-          if (slot >= 0 && slot < a.n_slots) v[i] = ((cnt + BN - 1) / BN) * FT;
+          if (slot >= 0 && slot < a.n_slots) rows = cnt;
           else if (slot != MOE_SLOT_SKIP) flag_error(a.err, MOE_DEVERR_NOT_RESIDENT);
         }
+        v[i] = (rows / BN) * FT;
+        sh.prow[e] = int16_t(rows % BN);
+        nparts += (rows % BN) != 0;
       }
       local += v[i];
     }
@@ -323,14 +361,32 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (e < E) sh.tstart[e] = run;
       run += v[i];
     }
-    if (lane == 31) { sh.tstart[E] = incl; sh.total_tiles = incl; sh.off[E] = a.offsets[E]; }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nparts += __shfl_xor_sync(0xffffffffu, nparts, o);
+    if (lane == 31) {
+      sh.tstart[E] = incl;
+      sh.full_tiles = incl;
+      sh.total_tiles = incl + nparts * FT;
+      sh.off[E] = a.offsets[E];
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid < E && sh.prow[tid] > 0) {  // rank of this expert's narrow tile: widest first, ties by index
+    const int mine = sh.prow[tid];
+    int rank = 0;
+    for (int e = 0; e < E; ++e) {
+      const int r = sh.prow[e];
+      rank += r > mine || (r == mine && e < tid);
+    }
+    sh.porder[rank] = int16_t(tid);
+  }
+  __syncthreads();
   const uint32_t tmem = sh.tmem_base;
   const int total = sh.total_tiles;
-  const int my_tiles = total > int(blockIdx.x) ? (total - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+  const int rounds = total / int(gridDim.x), rem = total % int(gridDim.x);
+  const int my_tiles = rounds + (rem > 0 && ((rounds & 1) ? int(gridDim.x) - 1 - int(blockIdx.x) : int(blockIdx.x)) < rem);
   const int iters = my_tiles * KS;
   uint8_t *const ringA = smem + C::A_OFF, *const ringB = smem + C::B_OFF, *const ringC = smem + C::C_OFF;
 
@@ -353,7 +409,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ks == KS || deq_tile < 0) {
         ks = 0;
         ++deq_tile;
-        const Tile tl = decode_tile<C::FW>(sh, E, FT, int(blockIdx.x) + deq_tile * int(gridDim.x));
+        const Tile tl = decode_tile<C::FW>(sh, E, FT, sched_pos(deq_tile));
         const int slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
         const uint8_t *rec = a.bank + int64_t(slot) * a.rec;
         // row of this thread's weights; down rows past H (a ragged last
@@ -429,8 +485,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = (warp - EPI_WARP0) >> 2;     // which quarter of the token columns
     const int frow = q * 32 + lane;                  // feature within the tile
     for (int tl_i = 0; tl_i < my_tiles; ++tl_i) {
-      const int t = int(blockIdx.x) + tl_i * int(gridDim.x);
-      const Tile tl = decode_tile<C::FW>(sh, E, FT, t);
+      const Tile tl = decode_tile<C::FW>(sh, E, FT, sched_pos(tl_i));
       const int b = tl_i % C::NBUF;
       const int f = tl.f0 + frow;
       if (!__all_sync(0xffffffffu, wait_bounded(sh, &sh.tmem_full[b], (tl_i / C::NBUF) & 1, a.err))) break;
@@ -448,9 +503,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int j_lo = quarter * (BN / 4), j_hi = min(tl.nvalid, j_lo + BN / 4);
       const int64_t row0 = int64_t(tl.lo + tl.n0);
       for (int j0 = j_lo; j0 < j_hi; j0 += 16) {
-        uint32_t g[16], u[16];  // gate/up: gate and up sums; down: the two 128-row output blocks
-        tmem_ld16x2(tbase + j0, tbase + BN + j0, g, u);
-        if (GATEUP) {
+        if constexpr (GATEUP) {
+          uint32_t g[16], u[16];  // gate and up sums of 16 tokens
+          tmem_ld16x2(tbase + j0, tbase + BN + j0, g, u);
           uint16_t *hp = a.h + (row0 + j0) * NOUT + f;
           bool bad = false;  // an h outside FP16's finite range cannot be the down pass's operand
 #pragma unroll
@@ -464,15 +519,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           if (bad) flag_error(a.err, MOE_DEVERR_RANGE);
         } else {
-          const uint32_t (&g2)[16] = u;  // second 128-row block
+          // the two 128-row output blocks one after the other (16 accumulator
+          // registers live instead of 32); the second block exists for the
+          // whole warp or for none of it: f0 is a multiple of 256 and H of 128
           float *yp = a.y + (row0 + j0) * NOUT + f;
+          uint32_t v[16];
+          tmem_ld16(tbase + j0, v);
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj)
-            if (j0 + jj < j_hi) yp[jj * NOUT] = __uint_as_float(g[jj]) * unscale0;
-          if (f + BM < NOUT) {
+            if (j0 + jj < j_hi) yp[jj * NOUT] = __uint_as_float(v[jj]) * unscale0;
+          if (tl.f0 + 2 * BM <= NOUT) {
+            tmem_ld16(tbase + BN + j0, v);
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj)
-              if (j0 + jj < j_hi) yp[jj * NOUT + BM] = __uint_as_float(g2[jj]) * unscale1;
+              if (j0 + jj < j_hi) yp[jj * NOUT + BM] = __uint_as_float(v[jj]) * unscale1;
           }
         }
       }
@@ -525,7 +585,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int it = 0; it < iters; ++it) {
       bool ok = true;
       if (ks == 0) {
-        const Tile tl = decode_tile<C::FW>(sh, E, FT, int(blockIdx.x) + tl_i * int(gridDim.x));
+        const Tile tl = decode_tile<C::FW>(sh, E, FT, sched_pos(tl_i));
         n16 = max(1, (tl.nvalid + 15) >> 4);
         ok = wait_bounded(sh, &sh.tmem_empty[tl_i % C::NBUF], ((tl_i / C::NBUF) & 1) ^ 1, a.err);
       }
@@ -553,7 +613,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (cur < 0 || ks == KS) {
         ks = 0;
         ++cur;
-        const Tile tl = decode_tile<C::FW>(sh, E, FT, int(blockIdx.x) + cur * int(gridDim.x));
+        const Tile tl = decode_tile<C::FW>(sh, E, FT, sched_pos(cur));
         slot = a.expert_slot ? a.expert_slot[tl.e] : tl.e;
         row_b = tl.lo + tl.n0;  // first activation row of the tile, in group order
         f0 = tl.f0;
