@@ -320,9 +320,10 @@ def measure_T(stack, T, steps, warmup, world, want_e2e=True, want_roofline=True)
         with torch.cuda.graph(g3, stream=stream):
             for l in range(stack.layers):
                 b = bufs[l]
-                M.moe_grouped_w4a16_ffn(x_in if l == 0 else xs[(l - 1) % 2], b.sorted_pair, b.offsets,
-                                        stack.banks[l].ptr, stack.banks[l].rec, None, stack.E, T, stack.K, stack.E,
-                                        stack.H, stack.I, b.path, b.y, b.ffn_ws, b.ffn_ws_bytes)
+                x_ffn, path = b.ffn_input(x_in if l == 0 else xs[(l - 1) % 2])
+                M.moe_grouped_w4a16_ffn(x_ffn, b.sorted_pair, b.offsets, stack.banks[l].ptr, stack.banks[l].rec,
+                                        None, stack.E, T, stack.K, stack.E, stack.H, stack.I, path, b.y, b.ffn_ws,
+                                        b.ffn_ws_bytes)
         ms_ffn_layers = time_graph(torch, g3, max(3, min(steps, 50)), 3)
         del g3
         n_act = [int((b.counts > 0).sum().item()) for b in bufs]
@@ -538,18 +539,18 @@ def slotcache_runs(layers, runs, steps, warmup):
             for l in range(L):
                 b = bufs[l]
                 b.topk_ids.copy_(ids_dev[si, l])
-                M.moe_route_topk(cur, stack.routers[l], T, H, E, K, None, M.MOE_IDS_GIVEN, b.logits, b.topk_ids,
-                                 b.topk_w)
+                M.moe_route_topk_x16(cur, stack.routers[l], T, H, E, K, None, M.MOE_IDS_GIVEN, b.logits,
+                                     b.topk_ids, b.topk_w, b.x16, b.ffn_ws)
                 M.moe_group_tokens(b.topk_ids, T, K, E, b.counts, b.offsets, b.sorted_pair, b.pair_pos,
                                    b.group_ws, b.group_ws_bytes)
+                x_ffn, path = b.ffn_input(cur)
                 waves = cache.plan_waves(l, [int(v) for v in routing[l][si].reshape(-1)])
                 n_waves[0] += len(waves)
                 for w in waves:
                     _, miss = cache.lookup(l, w)
                     cache.fill(l, miss, side=side, compute=comp)
-                    M.moe_grouped_w4a16_ffn(cur, b.sorted_pair, b.offsets, slots.data_ptr() + l * S * rec, rec,
-                                            table[l], S, T, K, E, H, I, M.MOE_PATH_AUTO, b.y, b.ffn_ws,
-                                            b.ffn_ws_bytes)
+                    M.moe_grouped_w4a16_ffn(x_ffn, b.sorted_pair, b.offsets, slots.data_ptr() + l * S * rec, rec,
+                                            table[l], S, T, K, E, H, I, path, b.y, b.ffn_ws, b.ffn_ws_bytes)
                     cache.release(l, comp)
                 out = xs[l % 2]
                 M.moe_combine(b.y, b.topk_w, b.pair_pos, cur, T, K, H, out)

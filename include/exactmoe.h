@@ -147,6 +147,24 @@ int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router,
                    moe_stream_t stream);
 
 /*
+ * moe_route_topk that also writes x16 [T][H], the FP16 copy of x that the
+ * grouped FFN multiplies (pass it to moe_grouped_w4a16_ffn with
+ * MOE_FFN_X_F16): for decode-sized T (<= 64) the router kernel converts the
+ * rows it has already staged, so the FFN needs no conversion pass of its own;
+ * otherwise a separate conversion kernel runs after the routing. x is
+ * required (also with MOE_LOGITS_GIVEN), x16 must be 16-byte aligned. A value
+ * v converts exactly when 2^-17 <= |v| <= 65504 or v = 0; smaller magnitudes
+ * round to a multiple of 2^-24; a larger one sets MOE_DEVERR_RANGE in *err
+ * (a device int32 error word, e.g. word 0 of the FFN workspace, which
+ * moe_read_device_error reads; NULL: not reported).
+ */
+int moe_route_topk_x16(const moe_bf16 *x, const moe_bf16 *w_router,
+                       int T, int H, int E, int k,
+                       const float *bias, int flags,
+                       moe_bf16 *logits, int32_t *topk_ids, float *topk_w,
+                       uint16_t *x16, int32_t *err, moe_stream_t stream);
+
+/*
  * A4 — group the T*k (token, slot) pairs by expert (Figure 1 caption: the
  * tokens are gathered per chosen expert).
  *   topk_ids    [T][k] int32.
@@ -207,6 +225,9 @@ int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E,
 #define MOE_PATH_SEQUENTIAL 3 /* reference only: the GEMV kernels launched
                                  once per expert, expert after expert (the
                                  pages' sequential W4 baseline, Abstract) */
+#define MOE_FFN_X_F16 0x100   /* flag OR-ed into the path: x holds the FP16
+                                 copy of the activations (moe_route_topk_x16)
+                                 instead of BF16, so no conversion pass runs */
 
 /*
  * A5 + A6 — the grouped SwiGLU expert FFN with in-kernel int4 dequantisation
@@ -216,7 +237,7 @@ int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E,
  * t = sorted_pair[r] / k:
  *   h[r] = bf16_rn(silu(x[t] Wg_e^T) * (x[t] Wu_e^T))      (fp32 sums)
  *   y[r] = h[r] Wd_e^T                                      (fp32 sums, fp32)
- *   x            [T][H] BF16.
+ *   x            [T][H] BF16, or FP16 when the path carries MOE_FFN_X_F16.
  *   bank         device array of expert records with stride record_bytes
  *                (moe_expert_record_layout(H, I).bytes or larger, multiple
  *                of 256).

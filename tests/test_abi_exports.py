@@ -73,6 +73,22 @@ def test_argument_checks_run_before_any_cuda_call(native):
     # T == 0 is a no-op that launches nothing
     assert lib.moe_combine(None, None, None, None, 0, 2, 2048, None, None) == native.MOE_OK
     assert lib.moe_route_topk(None, None, 0, 2048, 64, 8, None, 0, None, None, None, None) == native.MOE_OK
+    # the FP16-copy variant needs x and x16 (also with given logits) and H a multiple of 8
+    assert lib.moe_route_topk_x16(16, 16, 4, 2048, 64, 8, None, 0, 16, 16, 16, None, None, None) == \
+        native.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_topk_x16(None, 16, 4, 2048, 64, 8, None, 2, 16, 16, 16, 16, None, None) == \
+        native.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_topk_x16(16, 16, 4, 2044, 64, 8, None, 0, 16, 16, 16, 16, None, None) == \
+        native.MOE_ERR_SHAPE
+    assert lib.moe_route_topk_x16(16, 16, 4, 2048, 64, 8, None, 0, 16, 16, 16, 24, None, None) == \
+        native.MOE_ERR_INVALID_ARG  # x16 not 16-byte aligned
+    assert lib.moe_route_topk_x16(None, None, 0, 2048, 64, 8, None, 0, None, None, None, None, None, None) == \
+        native.MOE_OK
+    # the FP16-input flag is stripped before the path check, an unknown bit is not
+    assert lib.moe_grouped_w4a16_ffn(16, 16, 16, 256, 3244032, None, 64, 4, 8, 64, 2048, 1024, 0x100 | 7,
+                                     16, 256, 1 << 20, None) == native.MOE_ERR_INVALID_ARG
+    assert native.moe_ffn_workspace_size(16, 8, 64, 2048, 1024, 0x100 | 1) == \
+        native.moe_ffn_workspace_size(16, 8, 64, 2048, 1024, 1)
 
 
 def test_slot_cache_lru_matches_oracle(native):

@@ -191,7 +191,8 @@ def _make_bank(M, gate, up, down):
     return bank
 
 
-def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None):
+def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None, x16=None):
+    """x16: an FP16 copy of x passed with MOE_FFN_X_F16 instead of x."""
     T, H = x.shape
     I = bank.I
     d = torch.from_numpy(ids.astype(np.int32)).cuda()
@@ -205,8 +206,9 @@ def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None):
     nb = M.moe_ffn_workspace_size(T, k, E, H, I, path)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     es = None if expert_slot is None else torch.tensor(expert_slot, dtype=torch.int32, device="cuda")
-    M.moe_grouped_w4a16_ffn(x.cuda(), sp, offsets, bank.ptr, bank.rec, es, bank.n if n_slots is None else n_slots,
-                            T, k, E, H, I, path, y, ws, nb)
+    x_in, p_in = (x.cuda(), path) if x16 is None else (x16.cuda(), path | M.MOE_FFN_X_F16)
+    M.moe_grouped_w4a16_ffn(x_in, sp, offsets, bank.ptr, bank.rec, es, bank.n if n_slots is None else n_slots,
+                            T, k, E, H, I, p_in, y, ws, nb)
     code = M.moe_read_device_error(ws)
     # h is internal: the BF16-rounded value held in FP16 (exact) on both paths
     h = ws[256:256 + T * k * I * 2].view(torch.float16).view(T * k, I)
@@ -235,6 +237,74 @@ def test_grouped_ffn(M, path, E, H, I, T, k):
     ref_h, ref_y = o.grouped_ffn(x.double().numpy(), experts, sp, offsets, k)
     assert_bf16_close(h, ref_h, "h")
     assert_bf16_close(y, ref_y, "y")
+
+
+@pytest.mark.parametrize("path", ["gemv", "tc", "seq"])
+@pytest.mark.parametrize("E,H,I,T,k", [(64, 2048, 1024, 16, 8), (4, 512, 256, 300, 2), (6, 384, 640, 70, 3)])
+def test_grouped_ffn_fp16_input(M, path, E, H, I, T, k):
+    """MOE_FFN_X_F16: the FFN fed the FP16 copy of x computes bit for bit what
+    it computes from the BF16 x (the same FP16 operands, no conversion pass),
+    and so meets the oracle's bar too."""
+    P = {"gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC, "seq": M.MOE_PATH_SEQUENTIAL}[path]
+    rng = np.random.default_rng(E * H + T + 7)
+    gate = synth.normal_bf16((E, I, H), 0.02, 1100 + E)
+    up = synth.normal_bf16((E, I, H), 0.02, 2100 + E)
+    down = synth.normal_bf16((E, H, I), 0.02, 3100 + E)
+    x = synth.activations(T, H, seed=15)
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    bank = _make_bank(M, gate, up, down)
+    y, h, code = _ffn_gpu(M, bank, x, ids, k, P, E)
+    x16 = torch.from_numpy(x.double().numpy().astype(np.float16))  # numpy's RNE conversion, not the library's
+    y16, h16, code16 = _ffn_gpu(M, bank, x, ids, k, P, E, x16=x16)
+    assert code == 0 and code16 == 0
+    assert np.array_equal(y16, y) and np.array_equal(h16, h)
+    experts = o.LazyQuantizedExperts(torch_weights_source(gate, up, down), E, H, I)
+    counts, offsets, sp, pp = o.group_tokens(ids, E)
+    ref_h, ref_y = o.grouped_ffn(x.double().numpy(), experts, sp, offsets, k)
+    assert_bf16_close(y16, ref_y, "y from the FP16 input")
+
+
+@pytest.mark.parametrize("T,H,E,k,flags", [(1, 2048, 64, 8, 0), (16, 2048, 64, 8, 0), (64, 2048, 64, 8, 0),
+                                           (37, 4096, 8, 2, 0), (100, 2048, 64, 8, 0), (300, 1024, 64, 8, 0),
+                                           (16, 2048, 64, 8, 2), (100, 2048, 64, 8, 2)])
+def test_route_topk_x16(M, T, H, E, k, flags):
+    """moe_route_topk_x16 routes exactly as moe_route_topk and writes the FP16
+    copy of x: fused into the decode router kernel for T <= 64, a conversion
+    pass otherwise, and with given logits (flags 2) a conversion pass too."""
+    x = synth.activations(T, H, seed=21 + T)
+    wr = synth.router_weight(0, E, H)
+    given = flags & M.MOE_LOGITS_GIVEN
+    lg_in = torch.from_numpy(np.round(np.random.default_rng(T).normal(size=(T, E)) * 8) / 8).to(torch.bfloat16)
+    ref_logits, ref_ids, ref_w = _route_gpu(M, x, wr, k, flags=flags, logits_in=lg_in if given else None)
+    logits = lg_in.cuda() if given else torch.empty(T, E, dtype=torch.bfloat16, device="cuda")
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    x16 = torch.full((T, H), float("nan"), dtype=torch.float16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_route_topk_x16(x.cuda(), wr.cuda(), T, H, E, k, None, flags, logits, ids, w, x16, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(logits.cpu(), ref_logits)
+    assert np.array_equal(ids.cpu().numpy(), ref_ids)
+    assert np.array_equal(w.cpu().double().numpy(), ref_w)
+    want = x.double().numpy().astype(np.float16)  # numpy's RNE conversion of the BF16 values
+    assert np.array_equal(x16.cpu().numpy().view(np.uint16), want.view(np.uint16))
+
+
+@pytest.mark.parametrize("T", [16, 100])
+def test_route_topk_x16_flags_values_beyond_fp16(M, T):
+    H, E, k = 2048, 64, 8
+    x = synth.activations(T, H, seed=4)
+    x[T // 2, 77] = 1.0e5                      # beyond FP16's largest finite value
+    logits = torch.empty(T, E, dtype=torch.bfloat16, device="cuda")
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    x16 = torch.empty(T, H, dtype=torch.float16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_route_topk_x16(x.cuda(), synth.router_weight(0, E, H).cuda(), T, H, E, k, None, 0, logits, ids, w, x16,
+                         err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == M.MOE_DEVERR_RANGE
 
 
 @pytest.mark.parametrize("E,H,I,T,k", [(5, 256, 384, 13, 2), (64, 2048, 1024, 16, 8), (8, 4096, 1024, 9, 2),

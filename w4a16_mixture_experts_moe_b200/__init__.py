@@ -11,11 +11,11 @@ from __future__ import annotations
 import importlib
 
 _NATIVE_NAMES = {
-    "moe_last_error", "moe_abi_version", "moe_launch_counter", "moe_expert_record_layout", "moe_quantize_pack", "moe_route_topk",
+    "moe_last_error", "moe_abi_version", "moe_launch_counter", "moe_expert_record_layout", "moe_quantize_pack", "moe_route_topk", "moe_route_topk_x16",
     "moe_group_workspace_size", "moe_group_tokens", "moe_group_tokens_noalloc", "MOE_NOALLOC_MAX_PAIRS", "moe_ffn_workspace_size", "moe_grouped_w4a16_ffn",
     "moe_combine", "moe_read_device_error", "moe_debug_stall_next_tc_ffn", "SlotCache", "MoeError",
     "moe_pool_save", "moe_pool_file_info", "moe_pool_load",
-    "MOE_RENORM", "MOE_LOGITS_GIVEN", "MOE_IDS_GIVEN", "MOE_PATH_AUTO", "MOE_PATH_GEMV", "MOE_PATH_TC", "MOE_PATH_SEQUENTIAL", "MOE_SLOT_SKIP",
+    "MOE_RENORM", "MOE_LOGITS_GIVEN", "MOE_IDS_GIVEN", "MOE_PATH_AUTO", "MOE_PATH_GEMV", "MOE_PATH_TC", "MOE_PATH_SEQUENTIAL", "MOE_SLOT_SKIP", "MOE_FFN_X_F16",
     "moe_bf16_record_layout", "moe_bf16_ffn_workspace_size", "moe_grouped_bf16_ffn",
     "MOE_DEVERR_NONE", "MOE_DEVERR_EXPERT_ID", "MOE_DEVERR_NOT_RESIDENT", "MOE_DEVERR_TIMEOUT", "MOE_DEVERR_RANGE",
 }

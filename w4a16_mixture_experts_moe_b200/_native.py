@@ -26,6 +26,7 @@ MOE_DEVERR_NONE, MOE_DEVERR_EXPERT_ID, MOE_DEVERR_NOT_RESIDENT, MOE_DEVERR_TIMEO
 MOE_RENORM, MOE_LOGITS_GIVEN, MOE_IDS_GIVEN = 1, 2, 4
 MOE_PATH_AUTO, MOE_PATH_GEMV, MOE_PATH_TC, MOE_PATH_SEQUENTIAL = 0, 1, 2, 3
 MOE_SLOT_SKIP = -2
+MOE_FFN_X_F16 = 0x100
 
 _p = C.c_void_p
 _i = C.c_int
@@ -55,6 +56,7 @@ SIGNATURES = {
     "moe_expert_record_layout": (_i, [_i, _i, C.POINTER(moe_record_layout)]),
     "moe_quantize_pack": (_i, [_p, _i, _i, _i, _p, _i64, _p, _i64, _p]),
     "moe_route_topk": (_i, [_p, _p, _i, _i, _i, _i, _p, _i, _p, _p, _p, _p]),
+    "moe_route_topk_x16": (_i, [_p, _p, _i, _i, _i, _i, _p, _i, _p, _p, _p, _p, _p, _p]),
     "moe_group_workspace_size": (_sz, [_i, _i, _i]),
     "moe_group_tokens": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_group_tokens_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _p, _p, _p]),
@@ -143,6 +145,11 @@ def moe_quantize_pack(w, E, N, K, packed, packed_stride, scales, scales_stride, 
 def moe_route_topk(x, w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w, stream=None):
     _check(lib.moe_route_topk(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(bias), flags, _ptr(logits),
                               _ptr(topk_ids), _ptr(topk_w), _stream(stream)))
+
+
+def moe_route_topk_x16(x, w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w, x16, err=None, stream=None):
+    _check(lib.moe_route_topk_x16(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(bias), flags, _ptr(logits),
+                                  _ptr(topk_ids), _ptr(topk_w), _ptr(x16), _ptr(err), _stream(stream)))
 
 
 def moe_group_workspace_size(T, k, E) -> int:

@@ -22,6 +22,9 @@ void count_launches(int n);
 // Raises a kernel's dynamic shared-memory limit on the current device (once
 // per device and kernel; later calls are a lookup).
 int allow_dynamic_smem(const void *kernel, size_t bytes, const char *what);
+// Enqueues x [n8 * 8] BF16 -> x16 FP16 (programmatic dependent launch);
+// MOE_DEVERR_RANGE goes to *err (if not NULL) for a value beyond FP16's range.
+int launch_bf16_to_f16(const uint16_t *x, uint16_t *x16, int64_t n8, int32_t *err, cudaStream_t s, const char *what);
 
 static inline cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -45,6 +48,22 @@ __device__ __forceinline__ uint16_t f_to_bf16(float f) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Eight BF16 values -> eight FP16 values (round to nearest even); `bad` is
+// set if any lies outside FP16's finite range. Exact for 2^-17 <= |v| <=
+// 65504 and for zero; smaller magnitudes round to a multiple of 2^-24.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, bool &bad) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float lo = bf16_lo(in[c]), hi = bf16_hi(in[c]);
+    bad |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+    const __half2 hv = __floats2half2_rn(lo, hi);
+    out[c] = *reinterpret_cast<const uint32_t *>(&hv);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 // First writer wins; later codes are dropped.

@@ -12,19 +12,6 @@ static size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 // Average rows per expert at which the tensor-core path takes over.
 constexpr int TC_MIN_ROWS_PER_EXPERT = 32;
 
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, bool &bad) {
-  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-  uint32_t out[4];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const float lo = bf16_lo(in[c]), hi = bf16_hi(in[c]);
-    bad |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
-    const __half2 hv = __floats2half2_rn(lo, hi);
-    out[c] = *reinterpret_cast<const uint32_t *>(&hv);
-  }
-  return make_uint4(out[0], out[1], out[2], out[3]);
-}
-
 // x [T][H] BF16 -> FP16 copy, the decode path's gate/up input: exact for
 // BF16 values v with 2^-17 <= |v| <= 65504 and for zero; smaller magnitudes
 // round to a multiple of 2^-24 (absolute error at most 2^-25); values above
@@ -43,7 +30,9 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t *__restric
 // tensor-core gate/up pass then loads each token tile of an expert as one
 // contiguous block of rows. One warp per row (grid-stride over rows); each
 // lane issues all its loads of a pass before converting and storing, so a
-// row costs one round trip rather than one per 16-byte piece.
+// row costs one round trip rather than one per 16-byte piece. F16IN: x
+// already holds FP16 values, which are copied as they are.
+template <bool F16IN>
 __global__ void __launch_bounds__(256) gather_x_f16_kernel(const uint16_t *__restrict__ x,
                                                            const int32_t *__restrict__ sorted_pair, int k, int T,
                                                            int H8, int64_t P, uint16_t *__restrict__ xs,
@@ -66,7 +55,8 @@ __global__ void __launch_bounds__(256) gather_x_f16_kernel(const uint16_t *__res
       for (int u = 0; u < U; ++u) v[u] = c0 + 32 * u < H8 ? __ldg(src + c0 + 32 * u) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int u = 0; u < U; ++u)
-        if (c0 + 32 * u < H8) dst[c0 + 32 * u] = ok ? bf16x8_to_f16x8(v[u], bad) : make_uint4(0, 0, 0, 0);
+        if (c0 + 32 * u < H8)
+          dst[c0 + 32 * u] = !ok ? make_uint4(0, 0, 0, 0) : F16IN ? v[u] : bf16x8_to_f16x8(v[u], bad);
     }
   }
   if (bad) flag_error(err, MOE_DEVERR_RANGE);
@@ -81,13 +71,17 @@ int take_tc_stall() {
   return v > 0 ? 1 : 0;
 }
 
-int launch_x_to_f16(const FfnArgs &a, cudaStream_t s) {
-  const int64_t n8 = int64_t(a.T) * a.H / 8;
+int launch_bf16_to_f16(const uint16_t *x, uint16_t *x16, int64_t n8, int32_t *err, cudaStream_t s, const char *what) {
   const int64_t want = (n8 + 255) / 256, cap = 148 * 8;
   const int blocks = int(want < cap ? (want > 0 ? want : 1) : cap);
-  const cudaError_t e = launch_pdl(x_to_f16_kernel, dim3(blocks), dim3(256), 0, s, a.x, a.x16, n8, a.err);
-  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (x to fp16): %s", cudaGetErrorString(e));
-  return check_launch("moe_grouped_w4a16_ffn (x to fp16)");
+  const cudaError_t e = launch_pdl(x_to_f16_kernel, dim3(blocks), dim3(256), 0, s, x, x16, n8, err);
+  if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "%s (x to fp16): %s", what, cudaGetErrorString(e));
+  return check_launch(what);
+}
+
+int launch_x_to_f16(const FfnArgs &a, cudaStream_t s) {
+  if (a.x_f16) return MOE_OK;  // the caller's x is the FP16 copy already
+  return launch_bf16_to_f16(a.x, a.x16, int64_t(a.T) * a.H / 8, a.err, s, "moe_grouped_w4a16_ffn (x to fp16)");
 }
 
 int launch_gather_x_f16(const FfnArgs &a, cudaStream_t s) {
@@ -95,7 +89,10 @@ int launch_gather_x_f16(const FfnArgs &a, cudaStream_t s) {
   const int64_t want = (P + 7) / 8, cap = 148 * 16;  // 8 rows (warps) per block
   const int blocks = int(want < cap ? (want > 0 ? want : 1) : cap);
   const cudaError_t e =
-      launch_pdl(gather_x_f16_kernel, dim3(blocks), dim3(256), 0, s, a.x, a.sorted_pair, a.k, a.T, a.H / 8, P, a.xs, a.err);
+      a.x_f16 ? launch_pdl(gather_x_f16_kernel<true>, dim3(blocks), dim3(256), 0, s, a.x, a.sorted_pair, a.k, a.T,
+                           a.H / 8, P, a.xs, a.err)
+              : launch_pdl(gather_x_f16_kernel<false>, dim3(blocks), dim3(256), 0, s, a.x, a.sorted_pair, a.k, a.T,
+                           a.H / 8, P, a.xs, a.err);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_grouped_w4a16_ffn (gather x): %s", cudaGetErrorString(e));
   return check_launch("moe_grouped_w4a16_ffn (gather x)");
 }
@@ -119,6 +116,7 @@ static bool may_use_tc(int T, int k, int E, int path) {
 }  // namespace moe
 
 extern "C" size_t moe_ffn_workspace_size(int T, int k, int E, int H, int I, int path) {
+  path &= ~MOE_FFN_X_F16;
   if (T < 0 || k < 1 || I < 0 || H < 0) return moe::WS_HEADER;
   // header | h [T*k][I] 16-bit | x as FP16: [T][H] (GEMV) or [T*k][H] in group order (tensor cores)
   const size_t xrows = moe::may_use_tc(T, k, E, path) ? size_t(T) * size_t(k) : size_t(T);
@@ -137,6 +135,8 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
     return set_error(MOE_ERR_SHAPE, "moe_grouped_w4a16_ffn: H=%d I=%d must be positive multiples of 128", H, I);
   if (int64_t(T) * k > (int64_t(1) << 30))
     return set_error(MOE_ERR_SHAPE, "moe_grouped_w4a16_ffn: T*k too large");
+  const bool x_f16 = (path & MOE_FFN_X_F16) != 0;
+  path &= ~MOE_FFN_X_F16;
   if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_TC && path != MOE_PATH_SEQUENTIAL)
     return set_error(MOE_ERR_INVALID_ARG, "moe_grouped_w4a16_ffn: unknown path %d", path);
   moe_record_layout L;
@@ -165,9 +165,10 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
   a.off_gs = L.gate_s; a.off_us = L.up_s; a.off_ds = L.down_s;
   a.err = static_cast<int32_t *>(ws);
   a.h = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER);
-  a.x16 = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER +
-                                       round256(size_t(T) * size_t(k) * size_t(I) * 2));
-  a.xs = a.x16;
+  a.xs = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + WS_HEADER +
+                                      round256(size_t(T) * size_t(k) * size_t(I) * 2));
+  a.x_f16 = x_f16;
+  a.x16 = x_f16 ? const_cast<uint16_t *>(x) : a.xs;
   a.y = y;
   a.stall = 0;
   a.e0 = 0;

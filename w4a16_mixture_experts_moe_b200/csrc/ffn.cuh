@@ -26,6 +26,7 @@ struct FfnArgs {
   int32_t *err;   // device error word
   int stall;      // test hook: producers never publish a stage (bounded waits run out)
   int e0;         // first expert of the launch (blockIdx.y + e0; the sequential path launches one expert)
+  int x_f16;      // x already holds FP16 values (MOE_FFN_X_F16): x16 = x and no conversion pass
 };
 
 // Test hook state (moe_debug_stall_next_tc_ffn): number of tensor-core FFN

@@ -85,7 +85,8 @@ template <int TOK>
 __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
     route_topk_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, int T, int H, int E, int k,
                       const float *__restrict__ bias, int flags, uint16_t *__restrict__ logits,
-                      int32_t *__restrict__ topk_ids, float *__restrict__ topk_w) {
+                      int32_t *__restrict__ topk_ids, float *__restrict__ topk_w, uint16_t *__restrict__ x16,
+                      int32_t *err) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ float part[TOK][RT_MAX_EPC];  // this CTA's logits (as fp32 of the BF16 value)
   __shared__ float keys[MAX_E];                   // the token this CTA ranks
@@ -135,6 +136,19 @@ __global__ void __cluster_dims__(RT_CLUSTER, 1, 1) __launch_bounds__(RT_THREADS)
       }
     }
     __syncthreads();
+    if (x16) {
+      // the FP16 copy of the staged rows for the grouped FFN: the cluster's
+      // CTAs hold the same rows, so each writes its share of the 16-byte pieces
+      const int per = (chunks + RT_CLUSTER - 1) / RT_CLUSTER;
+      const int c_lo = rank * per, n_c = max(0, min(chunks, c_lo + per) - c_lo);
+      bool bad = false;
+      for (int q = threadIdx.x; q < nt * n_c; q += RT_THREADS) {
+        const int tt = q / n_c, c = c_lo + q % n_c;
+        reinterpret_cast<uint4 *>(x16 + int64_t(t0 + tt) * H)[c] =
+            bf16x8_to_f16x8(reinterpret_cast<const uint4 *>(xs + tt * H)[c], bad);
+      }
+      if (bad) flag_error(err, MOE_DEVERR_RANGE);
+    }
     for (int e = e_lo + warp; e < e_hi; e += RT_THREADS / 32) {
       float acc[TOK];
 #pragma unroll
@@ -309,10 +323,12 @@ __global__ void __launch_bounds__(256) topk_kernel(const uint16_t *__restrict__ 
 
 }  // namespace moe
 
-extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T, int H, int E, int k,
-                              const float *bias, int flags, moe_bf16 *logits, int32_t *topk_ids,
-                              float *topk_w, moe_stream_t stream) {
-  using namespace moe;
+namespace moe {
+// Both entry points: x16 (nullable) receives the FP16 copy of x, fused into
+// the decode-sized router kernel or as a conversion pass after the routing.
+static int route_impl(const moe_bf16 *x, const moe_bf16 *w_router, int T, int H, int E, int k, const float *bias,
+                      int flags, moe_bf16 *logits, int32_t *topk_ids, float *topk_w, uint16_t *x16, int32_t *err,
+                      moe_stream_t stream) {
   if (flags & ~(MOE_RENORM | MOE_LOGITS_GIVEN | MOE_IDS_GIVEN))
     return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk: unknown flag bits 0x%x", flags);
   if (T < 0 || E < 1 || E > MAX_E || k < 1 || k > E || k > MAX_K)
@@ -338,7 +354,9 @@ extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T
     e = launch_pdl(topk_kernel, dim3(unsigned((T + 7) / 8)), dim3(256), 0, as_stream(stream), logits, T, E, k, bias,
                    flags, topk_ids, topk_w);
     if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_route_topk: %s", cudaGetErrorString(e));
-    return check_launch("moe_route_topk");
+    const int st = check_launch("moe_route_topk");
+    if (st != MOE_OK || !x16) return st;
+    return launch_bf16_to_f16(x, x16, int64_t(T) * H / 8, err, as_stream(stream), "moe_route_topk_x16");
   }
   const bool small = T <= 64;  // decode-sized: 2 tokens per cluster
   const int tok = small ? 2 : 8;
@@ -352,10 +370,35 @@ extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T
   }
   const int64_t blocks = int64_t((T + tok - 1) / tok) * RT_CLUSTER;
   if (blocks > 0x7fffffffLL) return set_error(MOE_ERR_SHAPE, "moe_route_topk: T too large");
+  // the router kernel writes x16 only from rows it stages (not with given logits)
+  uint16_t *x16_fused = need_x ? x16 : nullptr;
   e = small ? launch_pdl(route_topk_kernel<2>, dim3(unsigned(blocks)), dim3(RT_THREADS), smem, as_stream(stream), x,
-                         w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w)
+                         w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w, x16_fused, err)
             : launch_pdl(route_topk_kernel<8>, dim3(unsigned(blocks)), dim3(RT_THREADS), smem, as_stream(stream), x,
-                         w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w);
+                         w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w, x16_fused, err);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_route_topk: %s", cudaGetErrorString(e));
-  return check_launch("moe_route_topk");
+  const int st = check_launch("moe_route_topk");
+  if (st != MOE_OK || !x16 || x16_fused) return st;
+  return launch_bf16_to_f16(x, x16, int64_t(T) * H / 8, err, as_stream(stream), "moe_route_topk_x16");
+}
+}  // namespace moe
+
+extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T, int H, int E, int k,
+                              const float *bias, int flags, moe_bf16 *logits, int32_t *topk_ids,
+                              float *topk_w, moe_stream_t stream) {
+  return moe::route_impl(x, w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w, nullptr, nullptr, stream);
+}
+
+extern "C" int moe_route_topk_x16(const moe_bf16 *x, const moe_bf16 *w_router, int T, int H, int E, int k,
+                                  const float *bias, int flags, moe_bf16 *logits, int32_t *topk_ids,
+                                  float *topk_w, uint16_t *x16, int32_t *err, moe_stream_t stream) {
+  using namespace moe;
+  if (H < 8 || H % 8)
+    return set_error(MOE_ERR_SHAPE, "moe_route_topk_x16: H=%d must be a positive multiple of 8", H);
+  if (T > 0 && (!x || !x16))
+    return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk_x16: x and x16 are required");
+  if (T > 0 && (!aligned(x, 16) || !aligned(x16, 16)))
+    return set_error(MOE_ERR_INVALID_ARG, "moe_route_topk_x16: x and x16 must be 16-byte aligned");
+  return route_impl(x, w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w, T > 0 ? x16 : nullptr, err,
+                    stream);
 }

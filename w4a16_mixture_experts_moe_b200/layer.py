@@ -77,6 +77,13 @@ class Bf16Bank:
             recs[:, off:off + n].copy_(w.contiguous().view(E, -1).view(torch.uint8))
 
 
+# Up to this many tokens the router kernel also writes the FP16 copy of x
+# that the grouped FFN multiplies (moe_route_topk_x16 + MOE_FFN_X_F16), so the
+# FFN call runs no conversion pass; larger batches convert inside the FFN
+# (gathered into group order for the tensor-core path).
+ROUTER_X16_MAX_T = 64
+
+
 class LayerBuffers:
     """Per-shape device buffers of one layer step (T tokens, top-k of E)."""
 
@@ -97,6 +104,12 @@ class LayerBuffers:
         self.group_ws = torch.zeros(self.group_ws_bytes, dtype=torch.uint8, **d)
         self.ffn_ws_bytes = N.moe_ffn_workspace_size(T, k, E, H, I, path)
         self.ffn_ws = torch.zeros(self.ffn_ws_bytes, dtype=torch.uint8, **d)
+        self.x16 = torch.empty(T, H, dtype=torch.float16, **d) if 0 < T <= ROUTER_X16_MAX_T else None
+
+    def ffn_input(self, x):
+        """(activations, path) for moe_grouped_w4a16_ffn after this buffer's
+        routing: the router's FP16 copy when it wrote one, else x itself."""
+        return (self.x16, self.path | N.MOE_FFN_X_F16) if self.x16 is not None else (x, self.path)
 
 
 def moe_layer_forward(x, w_router, bank: ExpertBank, buf: LayerBuffers, *, bias=None, flags=0,
@@ -104,11 +117,16 @@ def moe_layer_forward(x, w_router, bank: ExpertBank, buf: LayerBuffers, *, bias=
     """route -> group -> grouped FFN -> combine for x [T][H]; returns `out`."""
     T, k, E, H, I = buf.T, buf.k, buf.E, buf.H, buf.I
     out = buf.out if out is None else out
-    N.moe_route_topk(x, w_router, T, H, E, k, bias, flags, buf.logits, buf.topk_ids, buf.topk_w, stream)
+    if buf.x16 is not None:  # the router also writes the FFN's FP16 input; range errors go to the FFN's word
+        N.moe_route_topk_x16(x, w_router, T, H, E, k, bias, flags, buf.logits, buf.topk_ids, buf.topk_w,
+                             buf.x16, buf.ffn_ws, stream)
+    else:
+        N.moe_route_topk(x, w_router, T, H, E, k, bias, flags, buf.logits, buf.topk_ids, buf.topk_w, stream)
     N.moe_group_tokens(buf.topk_ids, T, k, E, buf.counts, buf.offsets, buf.sorted_pair, buf.pair_pos,
                        buf.group_ws, buf.group_ws_bytes, stream)
-    N.moe_grouped_w4a16_ffn(x, buf.sorted_pair, buf.offsets, bank.ptr, bank.rec, expert_slot,
-                            bank.n if n_slots is None else n_slots, T, k, E, H, I, buf.path, buf.y,
+    x_ffn, path = buf.ffn_input(x)
+    N.moe_grouped_w4a16_ffn(x_ffn, buf.sorted_pair, buf.offsets, bank.ptr, bank.rec, expert_slot,
+                            bank.n if n_slots is None else n_slots, T, k, E, H, I, path, buf.y,
                             buf.ffn_ws, buf.ffn_ws_bytes, stream)
     N.moe_combine(buf.y, buf.topk_w, buf.pair_pos, residual, T, k, H, out, stream)
     return out
