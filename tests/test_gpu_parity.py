@@ -219,9 +219,12 @@ def _ffn_gpu(M, bank, x, ids, k, path, E, expert_slot=None, n_slots=None, x16=No
 @pytest.mark.parametrize("E,H,I,T,k", [(5, 256, 384, 13, 2), (4, 512, 256, 40, 3), (64, 2048, 1024, 16, 8),
                                        (8, 4096, 1024, 9, 2), (4, 512, 256, 300, 2), (6, 384, 640, 700, 3),
                                        (64, 2048, 1024, 1, 8), (64, 2048, 1024, 64, 8),
-                                       (8, 1024, 1024, 40, 2), (4, 1024, 2048, 100, 2)])
+                                       (8, 1024, 1024, 40, 2), (4, 1024, 2048, 100, 2), (256, 512, 256, 5, 8),
+                                       (64, 2048, 1024, 4, 8)])
 def test_grouped_ffn(M, path, E, H, I, T, k):
-    """Both FFN paths, and the sequential per-expert reference, against the oracle."""
+    """Both FFN paths, and the sequential per-expert reference, against the oracle
+    (with fewer (token, expert) pairs than experts the GEMV grid is compact:
+    one row per possible active expert)."""
     P = {"gemv": M.MOE_PATH_GEMV, "tc": M.MOE_PATH_TC, "seq": M.MOE_PATH_SEQUENTIAL}[path]
     rng = np.random.default_rng(E * H + T)
     gate = synth.normal_bf16((E, I, H), 0.02, 1000 + E)

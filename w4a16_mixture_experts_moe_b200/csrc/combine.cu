@@ -1,14 +1,17 @@
 // A7 — router-weighted combine of the k expert outputs of each token, with
 // an optional residual: out[t] = bf16_rn(res[t] + sum_j w[t][j] * y[pos(t,j)]),
 // fp32 expert outputs, fp32 accumulation in increasing j (deterministic). A
-// CTA covers CB_THREADS * 8 hidden elements of one token (grid: tokens x hidden
+// CTA covers CB_THREADS * 4 hidden elements of one token (grid: tokens x hidden
 // slices, so a small decode batch still spreads over many SMs); each thread
-// owns 8 consecutive elements.
+// owns 4 consecutive elements and issues the loads of up to CB_J expert rows
+// before the first multiply-add, so a token costs one round trip to L2 per
+// CB_J rows instead of one per row.
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int CB_THREADS = 64;
+constexpr int CB_THREADS = 128;
+constexpr int CB_J = 8;
 
 __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const float *__restrict__ y,
                                                               const float *__restrict__ topk_w,
@@ -25,35 +28,39 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const float *__rest
     ps[threadIdx.x] = pair_pos[int64_t(t) * k + threadIdx.x];
   }
   __syncthreads();
-  {
-    const int c = blockIdx.y * CB_THREADS + threadIdx.x;
-    if (c >= H / 8) return;
-    float acc[8];
-    if (residual) {
-      const uint4 r = reinterpret_cast<const uint4 *>(residual + int64_t(t) * H)[c];
-      acc[0] = bf16_lo(r.x); acc[1] = bf16_hi(r.x); acc[2] = bf16_lo(r.y); acc[3] = bf16_hi(r.y);
-      acc[4] = bf16_lo(r.z); acc[5] = bf16_hi(r.z); acc[6] = bf16_lo(r.w); acc[7] = bf16_hi(r.w);
-    } else {
+  const int c = blockIdx.y * CB_THREADS + threadIdx.x;  // 4-element piece of the row
+  if (c >= H / 4) return;
+  float acc[4];
+  if (residual) {
+    const uint2 r = reinterpret_cast<const uint2 *>(residual + int64_t(t) * H)[c];
+    acc[0] = bf16_lo(r.x); acc[1] = bf16_hi(r.x); acc[2] = bf16_lo(r.y); acc[3] = bf16_hi(r.y);
+  } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    }
-#pragma unroll 4
-    for (int j = 0; j < k; ++j) {
-      const int pos = ps[j];
-      if (pos < 0) continue;
-      const float w = ws[j];
-      const float4 *src = reinterpret_cast<const float4 *>(y + int64_t(pos) * H) + 2 * c;
-      const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
-      acc[0] = fmaf(w, v0.x, acc[0]); acc[1] = fmaf(w, v0.y, acc[1]);
-      acc[2] = fmaf(w, v0.z, acc[2]); acc[3] = fmaf(w, v0.w, acc[3]);
-      acc[4] = fmaf(w, v1.x, acc[4]); acc[5] = fmaf(w, v1.y, acc[5]);
-      acc[6] = fmaf(w, v1.z, acc[6]); acc[7] = fmaf(w, v1.w, acc[7]);
-    }
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]); o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]); o.w = pack_bf16x2(acc[6], acc[7]);
-    reinterpret_cast<uint4 *>(out + int64_t(t) * H)[c] = o;
+    for (int i = 0; i < 4; ++i) acc[i] = 0.f;
   }
+  for (int j0 = 0; j0 < k; j0 += CB_J) {
+    float4 v[CB_J];
+#pragma unroll
+    for (int u = 0; u < CB_J; ++u) {
+      const int j = j0 + u;
+      const int pos = j < k ? ps[j] : -1;
+      v[u] = pos >= 0 ? __ldg(reinterpret_cast<const float4 *>(y + int64_t(pos) * H) + c)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < CB_J; ++u) {
+      const int j = j0 + u;
+      if (j < k && ps[j] >= 0) {  // dropped pairs contribute nothing, not even a zero
+        const float w = ws[j];
+        acc[0] = fmaf(w, v[u].x, acc[0]); acc[1] = fmaf(w, v[u].y, acc[1]);
+        acc[2] = fmaf(w, v[u].z, acc[2]); acc[3] = fmaf(w, v[u].w, acc[3]);
+      }
+    }
+  }
+  uint2 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  reinterpret_cast<uint2 *>(out + int64_t(t) * H)[c] = o;
 }
 
 }  // namespace moe
@@ -67,7 +74,7 @@ extern "C" int moe_combine(const float *y, const float *topk_w, const int32_t *p
   if (!y || !topk_w || !pair_pos || !out) return set_error(MOE_ERR_INVALID_ARG, "moe_combine: NULL pointer");
   if (!aligned(y, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)))
     return set_error(MOE_ERR_INVALID_ARG, "moe_combine: y, residual and out must be 16-byte aligned");
-  const dim3 grid(unsigned(T), unsigned((H / 8 + CB_THREADS - 1) / CB_THREADS));
+  const dim3 grid(unsigned(T), unsigned((H / 4 + CB_THREADS - 1) / CB_THREADS));
   cudaError_t e = launch_pdl(combine_kernel, grid, dim3(CB_THREADS), 0, as_stream(stream), y, topk_w, pair_pos,
                              residual, k, H, out);
   if (e != cudaSuccess) return set_error(MOE_ERR_CUDA, "moe_combine: %s", cudaGetErrorString(e));

@@ -172,6 +172,7 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
   a.y = y;
   a.stall = 0;
   a.e0 = 0;
+  a.compact = 0;
   if (T == 0) return MOE_OK;
   if (path == MOE_PATH_SEQUENTIAL) return launch_ffn_sequential(a, s);
 

@@ -27,6 +27,7 @@ struct FfnArgs {
   int stall;      // test hook: producers never publish a stage (bounded waits run out)
   int e0;         // first expert of the launch (blockIdx.y + e0; the sequential path launches one expert)
   int x_f16;      // x already holds FP16 values (MOE_FFN_X_F16): x16 = x and no conversion pass
+  int compact;    // GEMV grid row y = the y-th expert with rows (few pairs, many experts), not expert y
 };
 
 // Test hook state (moe_debug_stall_next_tc_ffn): number of tensor-core FFN
