@@ -46,10 +46,10 @@ SHAPES = {"olmoe": (2048, 1024, 64, 8), "wide": (4096, 14336, 8, 2)}   # (H, I, 
 
 # DRAM bytes (read + write) of one decode FFN call per active expert, from an
 # ncu capture of the shipped gate/up and down kernels (one-layer stack, T=16,
-# 53 active experts: gate/up 119.05 MB read + 2.98 MB written, down 59.75 MB
-# read + 0.06 MB written; 5.8 % above the 3,244,032 algorithmic bytes per
+# 53 active experts: gate/up 119.04 MB read + 2.97 MB written, down 59.76 MB
+# read + 0.08 MB written; 5.8 % above the 3,244,032 algorithmic bytes per
 # expert). Reported as roofline.traffic, scaled to the bench's active experts.
-DECODE_TRAFFIC_PER_ACTIVE_EXPERT = (119046656 + 2977024 + 59753472 + 58368) / 53
+DECODE_TRAFFIC_PER_ACTIVE_EXPERT = (119038464 + 2971648 + 59755776 + 76288) / 53
 
 # Prefill entries of the default line: (shape, T).
 PREFILL_CASES = (("olmoe", 2048), ("olmoe", 8192), ("wide", 8192))
