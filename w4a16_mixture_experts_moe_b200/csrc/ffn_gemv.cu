@@ -423,8 +423,18 @@ static cudaError_t launch_gemv_pair(const FfnArgs &a0, cudaStream_t s) {
   cudaError_t e = launch_pdl(gemv_gateup_kernel<KS>, g1, dim3(GV_WARPS * 32), 0, s, a);
   if (e != cudaSuccess) return e;
   count_launches(1);
-  dim3 g2((a.H + rows_per_cta * DOWN_RS - 1) / (rows_per_cta * DOWN_RS), ny);  // DOWN_RS slices per warp
-  e = launch_pdl(gemv_down_kernel<KS>, g2, dim3(GV_WARPS * 32), 0, s, a);
+  // the down pass splits K half as far as gate/up when KS = 4 on a full grid
+  // (a four-token step: 0.655 -> 0.636 ms); at one token, and at KS = 2, the
+  // same split as gate/up measured best (halving it: 0.403 -> 0.429 ms at
+  // T = 1, and 1.388 -> 1.434 ms at T = 64)
+  if (KS == 4 && !a.compact) {
+    const int rpd = (GV_WARPS / 2) * 16;
+    dim3 g2((a.H + rpd * DOWN_RS - 1) / (rpd * DOWN_RS), ny);  // DOWN_RS slices per warp
+    e = launch_pdl(gemv_down_kernel<2>, g2, dim3(GV_WARPS * 32), 0, s, a);
+  } else {
+    dim3 g2((a.H + rows_per_cta * DOWN_RS - 1) / (rows_per_cta * DOWN_RS), ny);  // DOWN_RS slices per warp
+    e = launch_pdl(gemv_down_kernel<KS>, g2, dim3(GV_WARPS * 32), 0, s, a);
+  }
   if (e == cudaSuccess) count_launches(1);
   return e;
 }
