@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const float *__rest
 
 extern "C" int moe_combine(const float *y, const float *topk_w, const int32_t *pair_pos,
                            const moe_bf16 *residual, int T, int k, int H, moe_bf16 *out, moe_stream_t stream) {
+  moe::NvtxScope nvtx_scope("moe_combine");
   using namespace moe;
   if (T < 0 || k < 1 || k > MAX_K || H < 8 || H % 8)
     return set_error(MOE_ERR_SHAPE, "moe_combine: T=%d k=%d H=%d (need T>=0, 1<=k<=32, H a multiple of 8)", T, k, H);

@@ -9,6 +9,8 @@
 
 #include <utility>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/exactmoe.h"
 
 namespace moe {
@@ -27,6 +29,16 @@ int allow_dynamic_smem(const void *kernel, size_t bytes, const char *what);
 int launch_bf16_to_f16(const uint16_t *x, uint16_t *x16, int64_t n8, int32_t *err, cudaStream_t s, const char *what);
 
 static inline cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// A named NVTX range over an entry point's host work (argument checks and
+// launches), so a timeline profiler shows each call of the layer step; a
+// no-op unless a profiler is attached.
+struct NvtxScope {
+  explicit NvtxScope(const char *name) { nvtxRangePushA(name); }
+  ~NvtxScope() { nvtxRangePop(); }
+  NvtxScope(const NvtxScope &) = delete;
+  NvtxScope &operator=(const NvtxScope &) = delete;
+};
 
 static inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -127,6 +127,7 @@ extern "C" int moe_grouped_w4a16_ffn(const moe_bf16 *x, const int32_t *sorted_pa
                                      const void *bank, int64_t record_bytes, const int32_t *expert_slot,
                                      int n_slots, int T, int k, int E, int H, int I, int path, float *y,
                                      void *ws, size_t ws_bytes, moe_stream_t stream) {
+  moe::NvtxScope nvtx_scope("moe_grouped_w4a16_ffn");
   using namespace moe;
   if (T < 0 || E < 1 || E > MAX_E || k < 1 || k > E || k > MAX_K)
     return set_error(MOE_ERR_SHAPE, "moe_grouped_w4a16_ffn: T=%d E=%d k=%d (need T>=0, 1<=E<=256, 1<=k<=min(E,32))",

@@ -154,6 +154,7 @@ extern "C" size_t moe_bf16_ffn_workspace_size(int T, int k, int E, int H, int I)
 extern "C" int moe_grouped_bf16_ffn(const moe_bf16 *x, const int32_t *sorted_pair, const int32_t *offsets,
                                     const void *bank, int64_t record_bytes, int T, int k, int E, int H, int I,
                                     float *y, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  moe::NvtxScope nvtx_scope("moe_grouped_bf16_ffn");
   using namespace moe;
   if (T < 0 || E < 1 || E > MAX_E || k < 1 || k > E || k > MAX_K)
     return set_error(MOE_ERR_SHAPE, "moe_grouped_bf16_ffn: T=%d E=%d k=%d (need T>=0, 1<=E<=256, 1<=k<=min(E,32))",

@@ -197,6 +197,7 @@ extern "C" size_t moe_group_workspace_size(int T, int k, int E) {
 extern "C" int moe_group_tokens(const int32_t *topk_ids, int T, int k, int E, int32_t *counts, int32_t *offsets,
                                 int32_t *sorted_pair, int32_t *pair_pos, void *ws, size_t ws_bytes,
                                 moe_stream_t stream) {
+  moe::NvtxScope nvtx_scope("moe_group_tokens");
   using namespace moe;
   if (T < 0 || E < 1 || E > MAX_E || k < 1 || k > E || k > MAX_K)
     return set_error(MOE_ERR_SHAPE, "moe_group_tokens: T=%d E=%d k=%d (need T>=0, 1<=E<=256, 1<=k<=min(E,32))", T, E, k);
@@ -275,6 +276,7 @@ static int noalloc_scratch(cudaStream_t stream, void **out) {
 extern "C" int moe_group_tokens_noalloc(const int32_t *topk_ids, int T, int k, int E, int32_t *counts,
                                         int32_t *offsets, int32_t *sorted_pair, int32_t *pair_pos,
                                         moe_stream_t stream) {
+  moe::NvtxScope nvtx_scope("moe_group_tokens_noalloc");
   using namespace moe;
   if (T < 0 || k < 1 || int64_t(T) * k > MOE_NOALLOC_MAX_PAIRS)
     return set_error(MOE_ERR_SHAPE, "moe_group_tokens_noalloc: T*k = %lld pairs exceeds the fixed scratch limit of %d",

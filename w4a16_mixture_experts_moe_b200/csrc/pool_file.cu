@@ -83,6 +83,7 @@ static int read_header(FILE *f, const char *path, PoolHeader *h, const char *wha
 }  // namespace moe
 
 extern "C" int moe_pool_save(const char *path, const moe_pool_info *info, const void *pool) {
+  moe::NvtxScope nvtx_scope("moe_pool_save");
   using namespace moe;
   if (!path || !pool) return set_error(MOE_ERR_INVALID_ARG, "moe_pool_save: NULL pointer");
   int st = check_info(info, "moe_pool_save");
@@ -130,6 +131,7 @@ extern "C" int moe_pool_file_info(const char *path, moe_pool_info *info) {
 }
 
 extern "C" int moe_pool_load(const char *path, void *pool, size_t capacity, moe_pool_info *info) {
+  moe::NvtxScope nvtx_scope("moe_pool_load");
   using namespace moe;
   if (!path || !pool) return set_error(MOE_ERR_INVALID_ARG, "moe_pool_load: NULL pointer");
   FILE *f = fopen(path, "rb");

@@ -59,6 +59,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
 extern "C" int moe_quantize_pack(const moe_bf16 *w, int E, int N, int K, uint8_t *packed,
                                  int64_t packed_stride, moe_bf16 *scales, int64_t scales_stride,
                                  moe_stream_t stream) {
+  moe::NvtxScope nvtx_scope("moe_quantize_pack");
   using namespace moe;
   if (!w || !packed || !scales) return set_error(MOE_ERR_INVALID_ARG, "moe_quantize_pack: NULL pointer");
   if (E < 1 || N < 1 || K < GROUP || K % GROUP)

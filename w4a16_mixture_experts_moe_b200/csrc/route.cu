@@ -386,12 +386,14 @@ static int route_impl(const moe_bf16 *x, const moe_bf16 *w_router, int T, int H,
 extern "C" int moe_route_topk(const moe_bf16 *x, const moe_bf16 *w_router, int T, int H, int E, int k,
                               const float *bias, int flags, moe_bf16 *logits, int32_t *topk_ids,
                               float *topk_w, moe_stream_t stream) {
+  moe::NvtxScope nvtx_scope("moe_route_topk");
   return moe::route_impl(x, w_router, T, H, E, k, bias, flags, logits, topk_ids, topk_w, nullptr, nullptr, stream);
 }
 
 extern "C" int moe_route_topk_x16(const moe_bf16 *x, const moe_bf16 *w_router, int T, int H, int E, int k,
                                   const float *bias, int flags, moe_bf16 *logits, int32_t *topk_ids,
                                   float *topk_w, uint16_t *x16, int32_t *err, moe_stream_t stream) {
+  moe::NvtxScope nvtx_scope("moe_route_topk_x16");
   using namespace moe;
   if (H < 8 || H % 8)
     return set_error(MOE_ERR_SHAPE, "moe_route_topk_x16: H=%d must be a positive multiple of 8", H);

@@ -120,6 +120,7 @@ static void rollback(moe_slot_cache *c, int layer) {
 
 extern "C" int slot_cache_lookup(moe_slot_cache *c, int layer, const int32_t *ids, int n, int32_t *slot_of_id,
                                  int32_t *miss_ids, int *n_miss) {
+  moe::NvtxScope nvtx_scope("slot_cache_lookup");
   using namespace moe;
   if (!c || !n_miss || (n > 0 && (!ids || !slot_of_id || !miss_ids)))
     return set_error(MOE_ERR_INVALID_ARG, "slot_cache_lookup: NULL pointer");
@@ -197,6 +198,7 @@ static int ensure_events(moe_slot_cache *c, int layer) {
 
 extern "C" int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss_ids, int n_miss, moe_stream_t side,
                                moe_stream_t compute) {
+  moe::NvtxScope nvtx_scope("slot_cache_fill");
   using namespace moe;
   if (!c || (n_miss > 0 && !miss_ids)) return set_error(MOE_ERR_INVALID_ARG, "slot_cache_fill: NULL pointer");
   if (layer < 0 || layer >= c->layers || n_miss < 0)
@@ -267,6 +269,7 @@ extern "C" int slot_cache_fill(moe_slot_cache *c, int layer, const int32_t *miss
 
 extern "C" int slot_cache_plan_waves(moe_slot_cache *c, int layer, const int32_t *ids, int n,
                                      int32_t *wave_ids, int32_t *wave_start, int *n_waves) {
+  moe::NvtxScope nvtx_scope("slot_cache_plan_waves");
   using namespace moe;
   if (!c || !n_waves || (n > 0 && (!ids || !wave_ids || !wave_start)))
     return set_error(MOE_ERR_INVALID_ARG, "slot_cache_plan_waves: NULL pointer");
@@ -301,6 +304,7 @@ extern "C" int slot_cache_plan_waves(moe_slot_cache *c, int layer, const int32_t
 }
 
 extern "C" int slot_cache_release(moe_slot_cache *c, int layer, moe_stream_t compute) {
+  moe::NvtxScope nvtx_scope("slot_cache_release");
   using namespace moe;
   if (!c || layer < 0 || layer >= c->layers) return set_error(MOE_ERR_INVALID_ARG, "slot_cache_release: bad argument");
   if (c->simulate) return MOE_OK;
