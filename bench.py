@@ -52,7 +52,9 @@ SHAPES = {"olmoe": (2048, 1024, 64, 8), "wide": (4096, 14336, 8, 2)}   # (H, I, 
 DECODE_TRAFFIC_PER_ACTIVE_EXPERT = (119038464 + 2971648 + 59755776 + 76288) / 53
 
 # Prefill entries of the default line: (shape, T).
-PREFILL_CASES = (("olmoe", 2048), ("olmoe", 8192), ("wide", 8192))
+# (shape, T, Zipf-skewed routing): every prefill configuration of the workload
+PREFILL_CASES = (("olmoe", 512, False), ("olmoe", 2048, False), ("olmoe", 8192, False), ("wide", 512, False),
+                 ("wide", 2048, False), ("wide", 8192, False), ("olmoe", 512, True))
 
 
 def rec_bytes(h, i):
@@ -425,8 +427,9 @@ def main():
     torch.cuda.empty_cache()
     prefill = {}
     if not a.no_prefill:
-        for shape, Tp in PREFILL_CASES:
-            prefill[f"{shape}-T{Tp}"] = prefill_entry(a, shape, Tp, rank, world, P)
+        for shape, Tp, skew in PREFILL_CASES:
+            key = f"{shape}-T{Tp}" + ("-zipf1.2-skew" if skew else "")
+            prefill[key] = prefill_entry(a, shape, Tp, rank, world, P, skew=skew)
             torch.cuda.empty_cache()
     slot = {}
     if not a.no_slotcache:
@@ -736,8 +739,8 @@ def prefill_entry(a, shape, T, rank, world, P, skew=False):
            "ms_per_step": r["ms_per_step"], "steps": steps,
            "e2e": {"value": replica_value(T, world, r["ms_e2e"]), "unit": "layer-tokens/s",
                    "h2d_bytes_per_step": T * H_ * 2, "d2h_bytes_per_step": T * H_ * 2},
-           "config": {"workload": f"{shape}-prefill", "T": T, "layers": 1, "H": H_, "I": I_, "E": E_, "k": K_,
-                      "renorm": renorm,
+           "config": {"workload": f"{shape}-prefill" + ("-zipf1.2-skew" if skew else ""), "T": T, "layers": 1,
+                      "H": H_, "I": I_, "E": E_, "k": K_, "renorm": renorm,
                       "l2": f"inputs larger than L2 ({E_ * rec_bytes(H_, I_) / 1e6:.0f} MB of packed experts "
                             f"+ {T * H_ * 2 / 1e6:.0f} MB of activations)"},
            "roofline": {"bound": "tensor", "kernel": "moe_grouped_w4a16_ffn (tcgen05 gate/up + down), per call",
@@ -748,6 +751,10 @@ def prefill_entry(a, shape, T, rank, world, P, skew=False):
                         "ms_per_call": r["ffn_ms_per_call"], "n_active_mean": r["n_active_mean"]},
            "gpu_launches": r["launches_per_step"] * steps,
            "clocks": r["clocks"]}
+    if skew:  # the load imbalance the skewed router produces in layer 0
+        counts = r["counts_layer0"]
+        ent["groups"] = {"largest": max(counts), "empty": sum(1 for c in counts if c == 0),
+                         "active": sum(1 for c in counts if c > 0)}
     ent["cpu_baseline"] = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         v, cores, desc = oracle_sample(T, seconds=5.0, shape=shape, tokens=64, skew=skew, renorm=renorm)
