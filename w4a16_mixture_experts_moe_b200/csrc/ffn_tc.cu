@@ -8,7 +8,8 @@
 // list built on the device from the group offsets), three rings of
 // shared-memory buffers, each k-step taking one slot of each:
 //   codes  the packed int4 codes of the tile's 128 weight rows (per matrix),
-//          small, so the ring runs 6-8 k-steps ahead of the MMA;
+//          3 slots of 8 KB, refilled as soon as the dequant warps hold a
+//          slot's codes in registers;
 //   B      256 FP16 activation rows (gate/up: x gathered into group order by
 //          a pre-pass; down: h), 128-byte-swizzled K-major as the MMA reads;
 //   A      the dequantised FP16 weights q*s, same swizzled layout.
